@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Throughput of the exact-attention hot path on B200 (libfa2).
+
+One step = the whole path on one batch: fa2_fwd, fa2_bwd_preprocess and
+fa2_bwd on B=8, H=16, N=2048, d=128, bf16, non-causal, synthetic N(0,1)
+inputs.  FLOPs per step count 4*B*H*N^2*d for the forward and 2.5x that for
+the backward (causal would halve both).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--sweep]
+
+Prints ONE JSON line (rank 0).  With --gpus N > 1 it must be launched under
+torchrun: every rank runs its own independent batch (the path shards over
+independent (batch, head) problems with no data exchange), the timed region
+is bracketed by barriers, and the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the plain definition of
+attention) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd+bwd TFLOP/s (bf16, hd128) vs N and % of B200 dense BF16 peak"
+WORKLOAD = dict(B=8, H=16, N=2048, d=128, causal=False)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def flops_fwd(B, H, N, d, causal=False):
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ dist
+def dist_setup(n_gpus):
+    import torch
+    if n_gpus <= 1 and "WORLD_SIZE" not in os.environ:
+        return 0, 1, 0
+    import datetime
+
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample(seconds: float, w):
+    """Time the fp64 oracle (fwd + bwd of whole heads) for about `seconds`."""
+    import numpy as np
+    import torch
+
+    from exact_attention_147_b200 import workloads as W
+    from oracle import attention as oa
+
+    wl = W.Workload("bench", B=1, N=w["N"], H=2, d=w["d"], causal=w["causal"], seed=100)
+    q, k, v, do = W.make_inputs(wl, "cpu")
+    heads = 0
+    t0 = time.perf_counter()
+    while True:
+        h = heads % 2
+        args = [t[0, :, h].to(torch.float64).numpy() for t in (q, k, v, do)]
+        oa.head_forward(*args[:3], wl.softmax_scale, w["causal"])
+        oa.head_backward(*args, wl.softmax_scale, w["causal"])
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    per_head = flops_fwd(1, 1, w["N"], w["d"], w["causal"]) * 3.5
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": per_head * heads / el / 1e12, "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{heads} whole heads (N={w['N']}, d={w['d']}) fwd+bwd in fp64, "
+                      f"{el:.1f} s", "seconds": el, "heads": heads}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = dict(WORKLOAD)
+    per_step = []
+    for _ in range(args.warmup):
+        oracle_sample(0.0, w)
+    t_total = 0.0
+    heads_total = 0
+    for _ in range(args.steps):
+        r = oracle_sample(2.0, w)
+        per_step.append(r)
+        t_total += r["seconds"]
+        heads_total += r["heads"]
+    per_head = flops_fwd(1, 1, w["N"], w["d"]) * 3.5
+    value = per_head * heads_total / t_total / 1e12
+    full_step_flops = flops_fwd(w["B"], w["H"], w["N"], w["d"]) * 3.5
+    cores = per_step[-1]["cores"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": full_step_flops / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "B=8 H=16 N=2048 d=128 non-causal fwd+bwd", **w,
+                   "sample": "each step times the oracle on whole heads of the workload "
+                             "(about 2 s); ms_per_step extrapolates to all B*H heads"},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{heads_total} heads fwd+bwd over {args.steps} steps"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args):
+    import torch
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    from exact_attention_147_b200 import fa2 as F
+    from exact_attention_147_b200 import workloads as W
+
+    F.load_library()
+    w = dict(WORKLOAD)
+    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+    wl = W.Workload("bench", B=B, N=N, H=H, d=d, causal=causal, seed=1000 + rank)
+    q, k, v, do = W.make_inputs(wl, "cuda")
+    out = torch.empty_like(q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    D = torch.empty_like(lse)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(1, F.workspace_size(B, N, H, d, torch.bfloat16)), dtype=torch.uint8,
+                     device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        F.fwd(q, k, v, None, causal, (-1, -1), None, 0.0, out=out, lse=lse)
+        if ev:
+            ev[1].record(stream)
+        F.bwd_preprocess(out, do, D)
+        if ev:
+            ev[2].record(stream)
+        F.bwd(do, q, k, v, lse, D, None, causal, (-1, -1), None, 0.0, False, dq, dk, dv, ws)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert F.device_status() == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = F.kernel_launches()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    n1 = F.kernel_launches()
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = max_over_ranks(start.elapsed_time(stop), world)
+    status = F.device_status()
+    assert status == 0, f"device status {status}"
+
+    ms_fwd = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    ms_pre = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms_bwd = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    f_fwd = flops_fwd(B, H, N, d, causal)
+    f_step = 3.5 * f_fwd
+    ms_step = ms_total / args.steps
+    value = world * f_step / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end: pinned host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (out, dq, dk, dv)]
+        hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e_step():
+            for dst, src in ((q, hq), (k, hk), (v, hv), (do, hdo)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in zip(houts, (out, dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        for _ in range(max(1, args.warmup // 2)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        t2.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms_e2e = max_over_ranks(s2.elapsed_time(t2), world) / args.steps
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in houts) + hlse.numel() * 4
+        e2e = {"value": world * f_step / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+
+    peaks, peak_src = load_peaks()
+    sustained = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    burst = float(peaks["bf16_tflops"])
+    bwd_tflops = 2.5 * f_fwd / (ms_bwd * 1e-3) / 1e12
+    fwd_tflops = f_fwd / (ms_fwd * 1e-3) / 1e12
+    pre_bytes = 2 * B * N * H * d * 2 + B * H * N * 4
+    pre_gbs = pre_bytes / (ms_pre * 1e-3) / 1e9
+    dominant = "fa2_bwd" if ms_bwd >= ms_fwd else "fa2_fwd"
+    achieved = bwd_tflops if dominant == "fa2_bwd" else fwd_tflops
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get(dominant)
+        except Exception:
+            traffic = None
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+                "frac": achieved / sustained, "traffic": traffic, "kernel": dominant,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a "
+                               f"multi-step loop)",
+                "frac_of_burst_peak": achieved / burst}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "B=8 H=16 N=2048 d=128 bf16 non-causal fwd+bwd (per GPU)",
+                   "B": B, "H": H, "N": N, "d": d, "causal": causal,
+                   "l2": "inputs larger than L2 (q,k,v,o,dO,dq,dk,dv = 512 MiB + 128 MiB "
+                         "fp32 dQ accumulator per GPU, vs 126 MB L2)",
+                   "flops_per_step": f_step},
+        "roofline": roofline,
+        "calls": {"fa2_fwd": {"ms": ms_fwd, "tflops": fwd_tflops,
+                              "frac_sustained": fwd_tflops / sustained},
+                  "fa2_bwd_preprocess": {"ms": ms_pre, "GB/s": pre_gbs,
+                                         "frac_hbm": pre_gbs / float(peaks["hbm_gbs"])},
+                  "fa2_bwd": {"ms": ms_bwd, "tflops": bwd_tflops,
+                              "frac_sustained": bwd_tflops / sustained}},
+        "gpu_launches": int(n1 - n0),
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        try:
+            line["cpu_baseline"] = {k2: v2 for k2, v2 in oracle_sample(12.0, w).items()
+                                    if k2 in ("value", "unit", "cores", "kind", "sample")}
+        except Exception as ex:  # pragma: no cover
+            line["cpu_baseline"] = {"error": str(ex)}
+    if args.sweep and world == 1:
+        line["sweep"] = run_sweep(F, W, args)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_sweep(F, W, args):
+    """TFLOP/s of fwd and bwd (timed separately) over the sequence-length
+    sweep at 16384 tokens per batch, both head splits, causal and not."""
+    import torch
+    res = []
+    for d in (128, 64):
+        for n in W.SWEEP_N:
+            for causal in (False, True):
+                w = W.sweep(n, d, causal)
+                q, k, v, do = W.make_inputs(w, "cuda")
+                out, lse = F.fwd(q, k, v, causal=causal)
+                D = F.bwd_preprocess(out, do)
+                dq, dk, dv = F.bwd(do, q, k, v, lse, D, causal=causal)
+                ws = torch.empty(max(1, F.workspace_size(w.B, w.N, w.H, w.d, torch.bfloat16)),
+                                 dtype=torch.uint8, device="cuda")
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                for _ in range(3):
+                    F.fwd(q, k, v, causal=causal, out=out, lse=lse)
+                    F.bwd(do, q, k, v, lse, D, causal=causal, dq=dq, dk=dk, dv=dv, workspace=ws)
+                torch.cuda.synchronize()
+                reps = 10
+                ev[0].record()
+                for _ in range(reps):
+                    F.fwd(q, k, v, causal=causal, out=out, lse=lse)
+                ev[1].record()
+                for _ in range(reps):
+                    F.bwd(do, q, k, v, lse, D, causal=causal, dq=dq, dk=dk, dv=dv, workspace=ws)
+                ev[2].record()
+                torch.cuda.synchronize()
+                ff = flops_fwd(w.B, w.H, w.N, w.d, causal)
+                tf = ev[0].elapsed_time(ev[1]) / reps
+                tb = ev[1].elapsed_time(ev[2]) / reps
+                res.append({"N": n, "d": d, "H": w.H, "B": w.B, "causal": causal,
+                            "fwd_ms": tf, "fwd_tflops": ff / (tf * 1e-3) / 1e12,
+                            "bwd_ms": tb, "bwd_tflops": 2.5 * ff / (tb * 1e-3) / 1e12})
+                del q, k, v, do, out, lse, D, dq, dk, dv, ws
+                torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="libfa2", choices=["libfa2", "reference"])
+    ap.add_argument("--sweep", action="store_true", help="add the sequence-length sweep")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

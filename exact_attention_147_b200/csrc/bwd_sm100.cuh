@@ -1,0 +1,725 @@
+// Backward pass of exact attention on sm_100a tensor cores (tcgen05 + TMEM).
+//
+// The probabilities are recomputed from Q, K and the forward's per-row
+// log-sum-exp instead of being stored (explainer "AI基础 | Flash Attention",
+// "Backward pass": only O(N) statistics are kept and the scores are rebuilt
+// on chip).  With L = sum(O o dO), D_i = sum_c dO_ic O_ic and scale c:
+//     P  = exp(c S - LSE),   dV = P^T dO,   dP = dO V^T,
+//     dS = P o (dP - D),     dK = c dS^T Q,  dQ = c dS K.
+//
+// Kernel 1, fa2_bwd_dkdv_sm100_kernel: one CTA per 128-key block of one
+// (batch, head), parallel over key blocks (FlashAttention-2 abstract: work
+// split across thread blocks even within a head).  K_j and V_j stay in shared
+// memory; the query blocks that see them stream through a TMA ring.  Per query
+// block, with keys on the TMEM lanes:
+//     S^T  = K Q^T          (tcgen05, SS)       -> TMEM [0,128)
+//     dP^T = V dO^T         (tcgen05, SS)       -> TMEM [128,256)
+//     P^T  = exp2(S^T c log2e - LSE log2e)       (compute warps, -> bf16 over S^T)
+//     dV  += P^T dO         (tcgen05, A from TMEM)
+//     dS^T = P^T o (dP^T - D)                    (compute warps, -> bf16 over dP^T
+//                                                 and to shared memory)
+//     dK  += dS^T Q         (tcgen05, A from TMEM)
+//     dQ_i = dS K           (tcgen05, A = dS from shared memory, MN-major)
+//                           -> TMEM [128,128+d), added into an fp32 dQ
+//                              accumulator in global memory with vector
+//                              reductions (order of the adds is not fixed).
+// With `deterministic`, kernel 1 skips dQ and kernel 2 produces it.
+//
+// Kernel 2, fa2_bwd_dq_sm100_kernel: one CTA per 128-query block; it walks
+// the visible key blocks in ascending order, recomputes S, P, dP, dS with
+// queries on the TMEM lanes and accumulates dQ += dS K in TMEM, so every
+// element of dQ is summed in the same order on every run.
+//
+// Warp roles (both kernels): a TMA producer warp, a single-thread MMA issuer
+// warp and a compute warpgroup (one TMEM lane = one row per thread); kernel 1
+// adds a warpgroup that drains dQ from TMEM into global memory.
+#pragma once
+
+#include <math_constants.h>
+
+#include "attn_common.cuh"
+#include "fwd_sm100.cuh"
+#include "sm100_ptx.cuh"
+
+namespace fa2 {
+
+struct BwdParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;   // inputs, box {64,1,128,1}
+  CUtensorMap tm_dq, tm_dk, tm_dv;       // outputs (bf16), same boxes
+  const float* lse;                      // [B,H,N]
+  const float* dvec;                     // [B,H,N]
+  float* dq_accum;                       // [B,H,N,d] fp32 (kernel 1 with dQ)
+  const float* alibi;                    // [H] or null
+  int N, H, B;
+  int wl, wr;
+  int nblocks;                           // ceil(N / 128)
+  int heavy_first;
+  float scale;                           // softmax scale c
+  float scale_log2;                      // c * log2(e)
+  unsigned long long wait_ns;
+};
+
+template <int HD>
+struct BwdCfg {
+  static constexpr int TILE = 128 * HD * 2;          // one 128-row bf16 tile
+  static constexpr int Q_STAGES = 2;
+  static constexpr int DO_STAGES = HD == 128 ? 1 : 2;
+  static constexpr int DS_BYTES = 128 * 128 * 2;
+  static constexpr int SIDE_BYTES = 2 * 128 * 4;     // lse2 and D of one query block
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = TILE;
+  static constexpr int OFF_Q = 2 * TILE;
+  static constexpr int OFF_DO = OFF_Q + Q_STAGES * TILE;
+  static constexpr int OFF_DS = OFF_DO + DO_STAGES * TILE;
+  static constexpr int OFF_SIDE = OFF_DS + DS_BYTES;
+  static constexpr int OFF_BARS = OFF_SIDE + Q_STAGES * SIDE_BYTES;
+  // kv_full, Q full/empty, dO full/empty, s_full, dp_full, p_ready, ds_ready,
+  // dq_full, dq_free, acc_full, drain
+  static constexpr int NBARS = 1 + 2 * Q_STAGES + 2 * DO_STAGES + 8;
+  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16 + 1024;
+  static constexpr int THREADS = 320;
+};
+
+template <int HD>
+struct DqCfg {
+  static constexpr int TILE = 128 * HD * 2;
+  static constexpr int SLOTS = HD == 128 ? 4 : 8;    // K/V ring
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = TILE;
+  static constexpr int OFF_KV = 2 * TILE;
+  static constexpr int OFF_BARS = OFF_KV + SLOTS * TILE;
+  static constexpr int NBARS = 1 + 2 * SLOTS + 5;
+  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16 + 1024;
+  static constexpr int THREADS = 192;
+};
+
+namespace bwd_detail {
+constexpr float LOG2E = 1.44269504088896340736f;
+constexpr int SITE_BPROD = 0x500, SITE_BMMA = 0x600, SITE_BCOMP = 0x700, SITE_BRED = 0x800;
+constexpr int SITE_QPROD = 0x900, SITE_QMMA = 0xA00, SITE_QCOMP = 0xB00;
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// Writes 16 packed bf16x2 words (32 columns starting at column `col0`) of
+// row `row` into a 128-byte-swizzled tile of 128 rows x (64-column boxes).
+__device__ __forceinline__ void st_sw128_row32(uint8_t* tile, int row, int col0,
+                                               const uint32_t (&w)[16]) {
+  const int box = col0 / 64;
+  const int u0 = (col0 % 64) / 8;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint8_t* dst = tile + box * (128 * 128) + row * 128 + (((u0 + q4) ^ (row & 7)) * 16);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+  }
+}
+}  // namespace bwd_detail
+
+// ---------------------------------------------------------------------------
+// Kernel 1: dK, dV (and the atomically accumulated dQ when WITH_DQ)
+// ---------------------------------------------------------------------------
+template <int HD, bool ALIBI, bool WITH_DQ>
+__global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<HD>;
+  using namespace bwd_detail;
+  constexpr int QS = C::Q_STAGES, DS = C::DO_STAGES;
+  constexpr int NCH = HD / 64;
+  constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + HD;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sDO = smem + C::OFF_DO;
+  uint8_t* sDS = smem + C::OFF_DS;
+  float* sSide = reinterpret_cast<float*>(smem + C::OFF_SIDE);  // [QS][2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
+  const uint32_t b0 = smem_u32(bars);
+  const uint32_t kv_full = b0;
+  auto q_full = [&](int s) { return b0 + 8u * (1 + s); };
+  auto q_empty = [&](int s) { return b0 + 8u * (1 + QS + s); };
+  auto do_full = [&](int s) { return b0 + 8u * (1 + 2 * QS + s); };
+  auto do_empty = [&](int s) { return b0 + 8u * (1 + 2 * QS + DS + s); };
+  const uint32_t s_full = b0 + 8u * (1 + 2 * QS + 2 * DS);
+  const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24;
+  const uint32_t dq_full = s_full + 32, dq_free = s_full + 40, acc_full = s_full + 48;
+  const uint32_t drain_bar = b0 + 8u * (C::NBARS - 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  AbortFlag ab{abort_flag};
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nhb = p.H * p.B;
+  int kb, hb;
+  if (p.heavy_first) {  // causal: key block 0 is seen by the most query blocks
+    kb = int(blockIdx.x / nhb);
+    hb = int(blockIdx.x % nhb);
+  } else {
+    kb = int(blockIdx.x % p.nblocks);
+    hb = int(blockIdx.x / p.nblocks);
+  }
+  const int h = hb % p.H, b = hb / p.H;
+  const int k0 = kb * 128;
+  const int k_last = min(p.N - 1, k0 + 127);
+  const int i_lo = p.wr >= 0 ? max(0, k0 - p.wr) : 0;
+  const int i_hi = p.wl >= 0 ? min(p.N - 1, k_last + p.wl) : p.N - 1;
+  const int qb_begin = i_lo / 128;
+  const int nq = i_hi / 128 - qb_begin + 1;
+  const size_t head_off = (size_t(b) * p.H + h) * p.N;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < C::NBARS; ++i) {
+      const uint32_t bar = b0 + 8u * i;
+      bar_init(bar, (bar == p_ready || bar == ds_ready || bar == dq_free) ? 128 : 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bar_arrive_expect_tx(kv_full, 2 * C::TILE);
+      for (int c = 0; c < NCH; ++c) {
+        tma_load_4d(smem_u32(sK + c * 16384), &p.tm_k, kv_full, c * 64, h, k0, b);
+        tma_load_4d(smem_u32(sV + c * 16384), &p.tm_v, kv_full, c * 64, h, k0, b);
+      }
+    }
+    int issued_q = 0, issued_do = 0;
+    bool ok = true;
+    for (int it = 0; it < nq && ok; ++it) {
+      const int i0 = (qb_begin + it) * 128;
+      const int sq = it % QS;
+      ok = wait_bar(q_empty(sq), ((it / QS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 0);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      // log2-scaled LSE and D of this query block, +inf / 0 past N
+      float* side = sSide + sq * 256;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = lane + 32 * e;
+        const int i = i0 + c;
+        float l2 = CUDART_INF_F, dv = 0.f;
+        if (i < p.N) {
+          const float l = p.lse[head_off + i];
+          l2 = l == -CUDART_INF_F ? CUDART_INF_F : l * LOG2E;
+          dv = p.dvec[head_off + i];
+        }
+        side[c] = l2;
+        side[128 + c] = dv;
+      }
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) {
+        bar_arrive_expect_tx(q_full(sq), C::TILE);
+        for (int c = 0; c < NCH; ++c)
+          tma_load_4d(smem_u32(sQ + sq * C::TILE + c * 16384), &p.tm_q, q_full(sq), c * 64, h, i0, b);
+      }
+      ++issued_q;
+      const int sd = it % DS;
+      ok = wait_bar(do_empty(sd), ((it / DS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (lane == 0) {
+        bar_arrive_expect_tx(do_full(sd), C::TILE);
+        for (int c = 0; c < NCH; ++c)
+          tma_load_4d(smem_u32(sDO + sd * C::TILE + c * 16384), &p.tm_do, do_full(sd), c * 64, h, i0,
+                      b);
+      }
+      ++issued_do;
+    }
+    if (lane == 0) {
+      drain_wait(kv_full, 0, p.wait_ns);
+      for (int k = max(0, issued_q - QS); k < issued_q; ++k) drain_wait(q_full(k % QS), (k / QS) & 1, p.wait_ns);
+      for (int k = max(0, issued_do - DS); k < issued_do; ++k)
+        drain_wait(do_full(k % DS), (k / DS) & 1, p.wait_ns);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_kq = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+      const uint32_t id_pd = idesc_bf16_f32(128, HD, 0, 1);   // dV, dK (B MN-major)
+      const uint32_t id_dq = idesc_bf16_f32(128, HD, 1, 1);   // dQ (A and B MN-major)
+      auto kmajor = [&](uint32_t d_tmem, const uint8_t* a, const uint8_t* bm) {
+        const uint32_t a0 = smem_u32(a), bb = smem_u32(bm);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          umma_ss(d_tmem, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024), id_kq, kk > 0);
+        }
+      };
+      auto from_tmem = [&](uint32_t d_tmem, uint32_t a_tmem, const uint8_t* bm, bool acc) {
+        const uint32_t bb = smem_u32(bm);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(bb + kk * 2048, 16384, 1024), id_pd,
+                  (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait_bar(kv_full, 0, ab, p.wait_ns, SITE_BMMA + 0);
+      if (ok) ok = wait_bar(q_full(0), 0, ab, p.wait_ns, SITE_BMMA + 1);
+      tc_fence_after();
+      if (ok) {
+        kmajor(tmem + T_S, sK, sQ);
+        umma_commit(s_full);
+      }
+      for (int it = 0; it < nq && ok; ++it) {
+        const int sq = it % QS, sd = it % DS;
+        ok = wait_bar(do_full(sd), (it / DS) & 1, ab, p.wait_ns, SITE_BMMA + 2);
+        if (ok && WITH_DQ && it > 0) ok = wait_bar(dq_free, (it - 1) & 1, ab, p.wait_ns, SITE_BMMA + 3);
+        if (!ok) break;
+        tc_fence_after();
+        kmajor(tmem + T_DP, sV, sDO + sd * C::TILE);                 // dP^T = V dO^T
+        umma_commit(dp_full);
+        ok = wait_bar(p_ready, it & 1, ab, p.wait_ns, SITE_BMMA + 4);
+        if (!ok) break;
+        tc_fence_after();
+        from_tmem(tmem + T_DV, tmem + T_S, sDO + sd * C::TILE, it > 0);  // dV += P^T dO
+        umma_commit(do_empty(sd));
+        if (it + 1 < nq) {
+          const int sn = (it + 1) % QS;
+          ok = wait_bar(q_full(sn), ((it + 1) / QS) & 1, ab, p.wait_ns, SITE_BMMA + 5);
+          if (!ok) break;
+          tc_fence_after();
+          kmajor(tmem + T_S, sK, sQ + sn * C::TILE);                // next S^T
+          umma_commit(s_full);
+        }
+        ok = wait_bar(ds_ready, it & 1, ab, p.wait_ns, SITE_BMMA + 6);
+        if (!ok) break;
+        tc_fence_after();
+        from_tmem(tmem + T_DK, tmem + T_DP, sQ + sq * C::TILE, it > 0);   // dK += dS^T Q
+        if (WITH_DQ) {
+          // dQ_i = dS K: A = dS (queries x keys) read MN-major from the dS^T
+          // tile, B = K (keys x d) MN-major.
+          const uint32_t a0 = smem_u32(sDS), kb0 = smem_u32(sK);
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            umma_ss(tmem + T_DP, sdesc_sw128(a0 + kk * 2048, 16384, 1024),
+                    sdesc_sw128(kb0 + kk * 2048, 16384, 1024), id_dq, kk > 0);
+        }
+        umma_commit(q_empty(sq));
+        if (WITH_DQ) umma_commit(dq_full);
+      }
+      umma_commit(acc_full);
+      umma_commit(drain_bar);
+      drain_wait(drain_bar, 0, p.wait_ns);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ compute (key rows)
+    const int r = warp * 32 + lane;
+    const int j = k0 + r;
+    int lo_q = p.wr >= 0 ? max(0, j - p.wr) : 0;
+    int hi_q = p.wl >= 0 ? min(p.N - 1, j + p.wl) : p.N - 1;
+    if (j >= p.N) {
+      lo_q = 1;
+      hi_q = 0;
+    }
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const float C2 = p.scale_log2;
+    float slope2 = 0.f;
+    if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
+    bool ok = true;
+    for (int it = 0; it < nq; ++it) {
+      const int i0 = (qb_begin + it) * 128;
+      const float* side = sSide + (it % QS) * 256;
+      ok = wait_bar(s_full, it & 1, ab, p.wait_ns, SITE_BCOMP + 0);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      float pr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + T_S + c * 32, u);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pr[c * 32 + e] = __uint_as_float(u[e]);
+      }
+      tmem_ld_wait();
+      const bool full = (i0 >= lo_q) && (i0 + 127 <= hi_q);
+      const float fj = float(i0 - j);
+#pragma unroll
+      for (int c = 0; c < 128; c += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(side + c);
+        float x0, x1, x2, x3;
+        if (ALIBI) {
+          x0 = fmaf(slope2, fabsf(fj + float(c)), fmaf(pr[c], C2, -l4.x));
+          x1 = fmaf(slope2, fabsf(fj + float(c + 1)), fmaf(pr[c + 1], C2, -l4.y));
+          x2 = fmaf(slope2, fabsf(fj + float(c + 2)), fmaf(pr[c + 2], C2, -l4.z));
+          x3 = fmaf(slope2, fabsf(fj + float(c + 3)), fmaf(pr[c + 3], C2, -l4.w));
+        } else {
+          x0 = fmaf(pr[c], C2, -l4.x);
+          x1 = fmaf(pr[c + 1], C2, -l4.y);
+          x2 = fmaf(pr[c + 2], C2, -l4.z);
+          x3 = fmaf(pr[c + 3], C2, -l4.w);
+        }
+        pr[c] = ex2(x0);
+        pr[c + 1] = ex2(x1);
+        pr[c + 2] = ex2(x2);
+        pr[c + 3] = ex2(x3);
+      }
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int i = i0 + c;
+          if (i < lo_q || i > hi_q) pr[c] = 0.f;
+        }
+      }
+      // P^T (bf16) over the first 64 columns of S^T, for dV += P^T dO
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = pack_bf16(pr[c * 32 + 2 * e], pr[c * 32 + 2 * e + 1]);
+        tmem_st16(tmem + lane_base + T_S + c * 16, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      bar_arrive(p_ready);
+      // dS^T = P^T o (dP^T - D), 32 columns at a time
+      ok = wait_bar(dp_full, it & 1, ab, p.wait_ns, SITE_BCOMP + 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + T_DP + c * 32, u);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int cc = c * 32 + 2 * e;
+          const float d0 = pr[cc] * (__uint_as_float(u[2 * e]) - side[128 + cc]);
+          const float d1 = pr[cc + 1] * (__uint_as_float(u[2 * e + 1]) - side[128 + cc + 1]);
+          w[e] = pack_bf16(d0, d1);
+        }
+        // columns already read: written below the read position
+        tmem_st16(tmem + lane_base + T_DP + c * 16, w);
+        if (WITH_DQ) st_sw128_row32(sDS, r, c * 32, w);
+      }
+      tmem_st_wait();
+      if (WITH_DQ) fence_proxy_async_smem();
+      tc_fence_before();
+      bar_arrive(ds_ready);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok) ok = wait_bar(acc_full, 0, ab, p.wait_ns, SITE_BCOMP + 2);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (ok) {
+      // dV and dK rows -> bf16 -> the V and K tiles (free now) -> TMA store
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t u[32], w[16];
+        tmem_ld32(tmem + lane_base + T_DV + c * 32, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+        st_sw128_row32(sV, r, c * 32, w);
+        tmem_ld32(tmem + lane_base + T_DK + c * 32, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16(__uint_as_float(u[2 * e]) * p.scale, __uint_as_float(u[2 * e + 1]) * p.scale);
+        st_sw128_row32(sK, r, c * 32, w);
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (ok && r == 0) {
+      for (int c = 0; c < NCH; ++c) {
+        tma_store_4d(&p.tm_dv, smem_u32(sV + c * 16384), c * 64, h, k0, b);
+        tma_store_4d(&p.tm_dk, smem_u32(sK + c * 16384), c * 64, h, k0, b);
+      }
+      bulk_commit();
+      bulk_wait_all();
+    }
+  } else if (WITH_DQ && warp < 8) {
+    // ------------------------------------------------------------ dQ drain (query rows)
+    const int q = (warp - 4) * 32 + lane;
+    const uint32_t lane_base = uint32_t((warp - 4) * 32) << 16;
+    for (int it = 0; it < nq; ++it) {
+      const int i = (qb_begin + it) * 128 + q;
+      bool ok = wait_bar(dq_full, it & 1, ab, p.wait_ns, SITE_BRED);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      float acc[HD];
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + T_DP + c * 32, u);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[c * 32 + e] = __uint_as_float(u[e]);
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      bar_arrive(dq_free);
+      if (i < p.N) {
+        float* dst = p.dq_accum + (head_off + i) * HD;
+#pragma unroll
+        for (int c = 0; c < HD; c += 4) red_add_v4(dst + c, acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 2: dQ by an ordered walk over key blocks (deterministic mode)
+// ---------------------------------------------------------------------------
+template <int HD, bool ALIBI>
+__global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_constant__ BwdParams p) {
+  using C = DqCfg<HD>;
+  using namespace bwd_detail;
+  constexpr int SLOTS = C::SLOTS;
+  constexpr int NCH = HD / 64;
+  constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sDO = smem + C::OFF_DO;
+  uint8_t* sKV = smem + C::OFF_KV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
+  const uint32_t b0 = smem_u32(bars);
+  const uint32_t qd_full = b0;
+  auto slot_full = [&](int s) { return b0 + 8u * (1 + s); };
+  auto slot_empty = [&](int s) { return b0 + 8u * (1 + SLOTS + s); };
+  const uint32_t s_full = b0 + 8u * (1 + 2 * SLOTS);
+  const uint32_t dp_full = s_full + 8, ds_ready = s_full + 16, acc_full = s_full + 24;
+  const uint32_t drain_bar = s_full + 32;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  AbortFlag ab{abort_flag};
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nhb = p.H * p.B;
+  int qb, hb;
+  if (p.heavy_first) {  // causal: the last query block sees the most keys
+    qb = p.nblocks - 1 - int(blockIdx.x / nhb);
+    hb = int(blockIdx.x % nhb);
+  } else {
+    qb = int(blockIdx.x % p.nblocks);
+    hb = int(blockIdx.x / p.nblocks);
+  }
+  const int h = hb % p.H, b = hb / p.H;
+  const int i0 = qb * 128;
+  const int i_last = min(p.N - 1, i0 + 127);
+  const int kv_lo = p.wl >= 0 ? max(0, i0 - p.wl) : 0;
+  const int kv_hi = p.wr >= 0 ? min(p.N - 1, i_last + p.wr) : p.N - 1;
+  const int kb_begin = kv_lo / 128;
+  const int nk = kv_hi / 128 - kb_begin + 1;
+  const size_t head_off = (size_t(b) * p.H + h) * p.N;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < C::NBARS; ++i) {
+      const uint32_t bar = b0 + 8u * i;
+      bar_init(bar, bar == ds_ready ? 128 : 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bar_arrive_expect_tx(qd_full, 2 * C::TILE);
+      for (int c = 0; c < NCH; ++c) {
+        tma_load_4d(smem_u32(sQ + c * 16384), &p.tm_q, qd_full, c * 64, h, i0, b);
+        tma_load_4d(smem_u32(sDO + c * 16384), &p.tm_do, qd_full, c * 64, h, i0, b);
+      }
+      int n = 0;
+      bool ok = true;
+      for (int it = 0; it < nk && ok; ++it) {
+        const int kv0 = (kb_begin + it) * 128;
+        for (int which = 0; which < 2; ++which, ++n) {
+          const int s = n % SLOTS;
+          if (!wait_bar(slot_empty(s), ((n / SLOTS) & 1) ^ 1, ab, p.wait_ns, SITE_QPROD)) {
+            ok = false;
+            break;
+          }
+          bar_arrive_expect_tx(slot_full(s), C::TILE);
+          const CUtensorMap* tm = which == 0 ? &p.tm_k : &p.tm_v;
+          for (int c = 0; c < NCH; ++c)
+            tma_load_4d(smem_u32(sKV + s * C::TILE + c * 16384), tm, slot_full(s), c * 64, h, kv0, b);
+        }
+      }
+      drain_wait(qd_full, 0, p.wait_ns);
+      for (int k = max(0, n - SLOTS); k < n; ++k) drain_wait(slot_full(k % SLOTS), (k / SLOTS) & 1, p.wait_ns);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_qk = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t id_dq = idesc_bf16_f32(128, HD, 0, 1);
+      auto kmajor = [&](uint32_t d_tmem, const uint8_t* a, const uint8_t* bm) {
+        const uint32_t a0 = smem_u32(a), bb = smem_u32(bm);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          umma_ss(d_tmem, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024), id_qk, kk > 0);
+        }
+      };
+      bool ok = wait_bar(qd_full, 0, ab, p.wait_ns, SITE_QMMA + 0);
+      int n = 0;
+      for (int it = 0; it < nk && ok; ++it, n += 2) {
+        const int sk = n % SLOTS, sv = (n + 1) % SLOTS;
+        ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_QMMA + 1);
+        if (!ok) break;
+        tc_fence_after();
+        kmajor(tmem + T_S, sQ, sKV + sk * C::TILE);     // S = Q K^T
+        umma_commit(s_full);
+        ok = wait_bar(slot_full(sv), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_QMMA + 2);
+        if (!ok) break;
+        tc_fence_after();
+        kmajor(tmem + T_DP, sDO, sKV + sv * C::TILE);   // dP = dO V^T
+        umma_commit(dp_full);
+        ok = wait_bar(ds_ready, it & 1, ab, p.wait_ns, SITE_QMMA + 3);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb0 = smem_u32(sKV + sk * C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)            // dQ += dS K
+          umma_ts(tmem + T_DQ, tmem + T_S + kk * 8, sdesc_sw128(kb0 + kk * 2048, 16384, 1024), id_dq,
+                  (it > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(slot_empty(sk));
+        umma_commit(slot_empty(sv));
+      }
+      umma_commit(acc_full);
+      umma_commit(drain_bar);
+      drain_wait(drain_bar, 0, p.wait_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ compute (query rows)
+    const int r = warp * 32 + lane;
+    const int i = i0 + r;
+    const int lo = p.wl >= 0 ? max(0, i - p.wl) : 0;
+    const int hi = i >= p.N ? -1 : (p.wr >= 0 ? min(p.N - 1, i + p.wr) : p.N - 1);
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const float C2 = p.scale_log2;
+    float lse2 = CUDART_INF_F, dval = 0.f, slope2 = 0.f;
+    if (i < p.N) {
+      const float l = p.lse[head_off + i];
+      lse2 = l == -CUDART_INF_F ? CUDART_INF_F : l * LOG2E;
+      dval = p.dvec[head_off + i];
+    }
+    if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
+    bool ok = true;
+    for (int it = 0; it < nk; ++it) {
+      const int kv0 = (kb_begin + it) * 128;
+      ok = wait_bar(s_full, it & 1, ab, p.wait_ns, SITE_QCOMP + 0);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      float pr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + T_S + c * 32, u);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pr[c * 32 + e] = __uint_as_float(u[e]);
+      }
+      tmem_ld_wait();
+      const float fi = float(i - kv0);
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        float x = fmaf(pr[c], C2, -lse2);
+        if (ALIBI) x = fmaf(slope2, fabsf(fi - float(c)), x);
+        pr[c] = ex2(x);
+      }
+      if (!(kv0 >= lo && kv0 + 127 <= hi)) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int j = kv0 + c;
+          if (j < lo || j > hi) pr[c] = 0.f;
+        }
+      }
+      ok = wait_bar(dp_full, it & 1, ab, p.wait_ns, SITE_QCOMP + 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + T_DP + c * 32, u);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int cc = c * 32 + 2 * e;
+          w[e] = pack_bf16(pr[cc] * (__uint_as_float(u[2 * e]) - dval),
+                           pr[cc + 1] * (__uint_as_float(u[2 * e + 1]) - dval));
+        }
+        tmem_st16(tmem + lane_base + T_S + c * 16, w);   // dS (bf16) over S
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      bar_arrive(ds_ready);
+    }
+    if (ok) ok = wait_bar(acc_full, 0, ab, p.wait_ns, SITE_QCOMP + 2);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (ok) {
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t u[32], w[16];
+        tmem_ld32(tmem + lane_base + T_DQ + c * 32, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16(__uint_as_float(u[2 * e]) * p.scale, __uint_as_float(u[2 * e + 1]) * p.scale);
+        st_sw128_row32(sQ, r, c * 32, w);   // Q tile is free once every MMA is done
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (ok && r == 0) {
+      for (int c = 0; c < NCH; ++c) tma_store_4d(&p.tm_dq, smem_u32(sQ + c * 16384), c * 64, h, i0, b);
+      bulk_commit();
+      bulk_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Zero-fill of the fp32 dQ accumulator (n4 float4 elements).
+__global__ void __launch_bounds__(256) zero_f32x4_kernel(float4* __restrict__ p, long long n4) {
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n4; i += (long long)gridDim.x * 256)
+    p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+}  // namespace fa2

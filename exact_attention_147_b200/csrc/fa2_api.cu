@@ -1,0 +1,420 @@
+// libfa2: the C ABI declared in include/fa2.h.
+//
+// Host side only: argument checks, TMA descriptor encoding, kernel choice and
+// launch on the caller's stream.  All arithmetic of the attention path runs
+// in the kernels included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <algorithm>
+#include <mutex>
+
+#include "../../include/fa2.h"
+#include "attn_common.cuh"
+#include "bwd_sm100.cuh"
+#include "fwd_sm100.cuh"
+#include "rowwise.cuh"
+#include "simt.cuh"
+#include "sm100_ptx.cuh"
+
+using namespace fa2;
+
+namespace {
+
+std::atomic<unsigned long long> g_wait_ns{1000ull * 1000ull * 1000ull};
+std::atomic<uint64_t> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+
+// ----------------------------------------------------------------- checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa2_status check_shape(int B, int N, int H, int d, fa2_dtype dtype) {
+  if (B < 1 || N < 1 || H < 1) return FA2_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA2_ERR_INVALID_ARG;
+  if (dtype != FA2_BF16 && dtype != FA2_F32) return FA2_ERR_INVALID_ARG;
+  // grid limits of the launches below
+  if (B > 65535 || H > 65535) return FA2_ERR_INVALID_ARG;
+  const long long pairs = (N + 255) / 256;
+  if (pairs * H * B > 0x7fffffffLL) return FA2_ERR_INVALID_ARG;
+  if ((long long)B * H * N > (1LL << 40)) return FA2_ERR_INVALID_ARG;
+  return FA2_OK;
+}
+
+fa2_status check_tensor(const void* p, const fa2_strides& s, fa2_dtype dtype) {
+  if (p == nullptr || !aligned16(p)) return FA2_ERR_INVALID_ARG;
+  const int64_t vec = dtype == FA2_BF16 ? 8 : 4;  // elements per 16 bytes
+  const int64_t lim = (int64_t(1) << 40) / (dtype == FA2_BF16 ? 2 : 4);
+  for (int64_t x : {s.b, s.n, s.h})
+    if (x < 1 || x % vec != 0 || x >= lim) return FA2_ERR_INVALID_ARG;
+  return FA2_OK;
+}
+
+fa2_status check_options(float softmax_scale, float dropout_p, const float* alibi) {
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale)) return FA2_ERR_INVALID_ARG;
+  if (std::isnan(dropout_p) || dropout_p < 0.f || dropout_p >= 1.f) return FA2_ERR_INVALID_ARG;
+  if (dropout_p != 0.f) return FA2_ERR_UNSUPPORTED;
+  if (alibi != nullptr && (reinterpret_cast<uintptr_t>(alibi) & 3u) != 0) return FA2_ERR_INVALID_ARG;
+  return FA2_OK;
+}
+
+#define FA2_TRY(expr)                 \
+  do {                                \
+    const fa2_status st_ = (expr);    \
+    if (st_ != FA2_OK) return st_;    \
+  } while (0)
+
+// ----------------------------------------------------------------- device
+struct DeviceInfo {
+  int sm_major = -1;
+  int sm_minor = -1;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+fa2_status current_device(int* dev, DeviceInfo* info) {
+  if (cudaGetDevice(dev) != cudaSuccess) return FA2_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return FA2_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[*dev];
+  if (di.sm_major < 0) {
+    if (cudaDeviceGetAttribute(&di.sm_major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&di.sm_minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess) {
+      di.sm_major = -1;
+      return FA2_ERR_CUDA;
+    }
+  }
+  *info = di;
+  return FA2_OK;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per
+// device.
+template <typename K>
+fa2_status ensure_smem(K kernel, int bytes, int dev, std::atomic<uint64_t>& done_mask) {
+  const uint64_t bit = uint64_t(1) << dev;
+  if (done_mask.load() & bit) return FA2_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return FA2_ERR_CUDA;
+  done_mask.fetch_or(bit);
+  return FA2_OK;
+}
+
+// ----------------------------------------------------------------- TMA
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+fa2_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::call_once(g_encode_once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  *fn = g_encode;
+  return g_encode ? FA2_OK : FA2_ERR_CUDA;
+}
+
+// 4-D map over a bf16 [B, N, H, d] tensor: dims (d, H, N, B), box
+// (64, 1, rows, 1), 128-byte swizzle; rows past N read as zeros and are not
+// written by stores.
+fa2_status encode_bf16_4d(CUtensorMap* m, const void* ptr, const fa2_strides& s, int B, int N, int H,
+                          int d, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  FA2_TRY(get_encoder(&enc));
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(s.h) * 2, cuuint64_t(s.n) * 2, cuuint64_t(s.b) * 2};
+  cuuint32_t box[4] = {64, 1, cuuint32_t(box_rows), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
+}
+
+Strides to_s(const fa2_strides& s) { return Strides{s.b, s.n, s.h}; }
+
+void normalise_window(int causal, int* wl, int* wr) {
+  if (*wl < 0) *wl = -1;
+  if (*wr < 0) *wr = -1;
+  if (causal) *wr = 0;  // causal: key j <= query i, the same as a right bound of 0
+  // (a right bound above 0 with causal still means j <= i)
+}
+
+float resolve_scale(float s, int d) { return s > 0.f ? s : 1.0f / std::sqrt(float(d)); }
+
+// Call after every group of `n` kernel launches.
+fa2_status launched(int n) {
+  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+  g_launches.fetch_add(uint64_t(n));
+  return FA2_OK;
+}
+
+std::atomic<uint64_t> g_smem_fwd128{0}, g_smem_fwd128a{0}, g_smem_fwd64{0}, g_smem_fwd64a{0};
+
+template <int HD, bool ALIBI>
+fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
+                            const fa2_strides& sv, const fa2_strides& so, int dev, int causal_order,
+                            cudaStream_t st, std::atomic<uint64_t>& mask) {
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  FA2_TRY(encode_bf16_4d(&p.tm_q, a.q, sq, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_bf16_4d(&p.tm_k, a.k, sk, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_bf16_4d(&p.tm_v, a.v, sv, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_bf16_4d(&p.tm_o, a.o, so, a.B, a.N, a.H, HD, 128));
+  p.lse = a.lse;
+  p.alibi = a.alibi;
+  p.N = a.N;
+  p.H = a.H;
+  p.B = a.B;
+  p.wl = a.wl;
+  p.wr = a.wr;
+  p.npairs = (a.N + 255) / 256;
+  p.heavy_first = causal_order;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.wait_ns = g_wait_ns.load();
+  auto kern = fa2_fwd_sm100_kernel<HD, ALIBI>;
+  constexpr int smem = FwdCfg<HD>::SMEM_BYTES;
+  FA2_TRY(ensure_smem(kern, smem, dev, mask));
+  const unsigned grid = unsigned(p.npairs) * unsigned(a.H) * unsigned(a.B);
+  kern<<<grid, FwdCfg<HD>::THREADS, smem, st>>>(p);
+  return launched(1);
+}
+
+template <int HD, bool ALIBI>
+fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
+                            const fa2_strides& sv, const fa2_strides& sdo, const fa2_strides& sdq,
+                            const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
+                            int dev, cudaStream_t st) {
+  static std::atomic<uint64_t> mask_dkdv{0}, mask_dkdv_nodq{0}, mask_dq{0};
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  FA2_TRY(encode_bf16_4d(&p.tm_q, a.q, sq, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_bf16_4d(&p.tm_k, a.k, sk, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_bf16_4d(&p.tm_v, a.v, sv, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_bf16_4d(&p.tm_do, a.dout, sdo, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_bf16_4d(&p.tm_dq, a.dq, sdq, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_bf16_4d(&p.tm_dk, a.dk, sdk, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_bf16_4d(&p.tm_dv, a.dv, sdv, a.B, a.N, a.H, HD, 128));
+  p.lse = a.lse;
+  p.dvec = a.dvec;
+  p.dq_accum = a.dq_accum;
+  p.alibi = a.alibi;
+  p.N = a.N;
+  p.H = a.H;
+  p.B = a.B;
+  p.wl = a.wl;
+  p.wr = a.wr;
+  p.nblocks = (a.N + 127) / 128;
+  p.heavy_first = (a.wr >= 0 || a.wl >= 0) ? 1 : 0;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.wait_ns = g_wait_ns.load();
+  const unsigned grid = unsigned(p.nblocks) * unsigned(a.H) * unsigned(a.B);
+  constexpr int smem1 = BwdCfg<HD>::SMEM_BYTES;
+  if (!deterministic) {
+    const long long n4 = (long long)a.B * a.H * a.N * HD / 4;
+    const unsigned zgrid = unsigned(std::min<long long>((n4 + 255) / 256, 148 * 16));
+    zero_f32x4_kernel<<<zgrid, 256, 0, st>>>(reinterpret_cast<float4*>(a.dq_accum), n4);
+    FA2_TRY(launched(1));
+    auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true>;
+    FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv));
+    k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
+    FA2_TRY(launched(1));
+    const long long rows = (long long)a.B * a.H * a.N;
+    const long long per_block = 256 / (HD / 4);
+    dq_convert_kernel<HD><<<unsigned((rows + per_block - 1) / per_block), 256, 0, st>>>(a);
+    return launched(1);
+  }
+  auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false>;
+  FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv_nodq));
+  k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
+  FA2_TRY(launched(1));
+  auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI>;
+  constexpr int smem2 = DqCfg<HD>::SMEM_BYTES;
+  FA2_TRY(ensure_smem(k2, smem2, dev, mask_dq));
+  k2<<<grid, DqCfg<HD>::THREADS, smem2, st>>>(p);
+  return launched(1);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa2_strerror(fa2_status s) {
+  switch (s) {
+    case FA2_OK: return "FA2_OK";
+    case FA2_ERR_INVALID_ARG: return "FA2_ERR_INVALID_ARG: invalid pointer, shape, stride or option";
+    case FA2_ERR_UNSUPPORTED: return "FA2_ERR_UNSUPPORTED: valid but not implemented";
+    case FA2_ERR_CUDA: return "FA2_ERR_CUDA: a CUDA call failed";
+    case FA2_ERR_DEVICE_TIMEOUT: return "FA2_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait";
+  }
+  return "unknown fa2_status";
+}
+
+uint64_t fa2_kernel_launches(void) { return g_launches.load(); }
+
+fa2_status fa2_set_wait_limit_ms(int ms) {
+  if (ms < 1) return FA2_ERR_INVALID_ARG;
+  g_wait_ns.store((unsigned long long)ms * 1000ull * 1000ull);
+  return FA2_OK;
+}
+
+fa2_status fa2_device_status(int* code, int clear) {
+  if (code == nullptr) return FA2_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA2_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fa2_device_status, sizeof(int)) != cudaSuccess) return FA2_ERR_CUDA;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_fa2_device_status, &zero, sizeof(int)) != cudaSuccess) return FA2_ERR_CUDA;
+  }
+  *code = v;
+  return v ? FA2_ERR_DEVICE_TIMEOUT : FA2_OK;
+}
+
+fa2_status fa2_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
+                   int H, int d, fa2_dtype dtype, fa2_strides sq, fa2_strides sk, fa2_strides sv,
+                   fa2_strides so, float softmax_scale, int causal, int window_left, int window_right,
+                   const float* alibi_slopes, float dropout_p, void* stream) {
+  FA2_TRY(check_shape(B, N, H, d, dtype));
+  FA2_TRY(check_tensor(q, sq, dtype));
+  FA2_TRY(check_tensor(k, sk, dtype));
+  FA2_TRY(check_tensor(v, sv, dtype));
+  FA2_TRY(check_tensor(o, so, dtype));
+  if (lse == nullptr || !aligned16(lse)) return FA2_ERR_INVALID_ARG;
+  if (o == q || o == k || o == v) return FA2_ERR_INVALID_ARG;
+  FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
+
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.alibi = alibi_slopes;
+  a.sq = to_s(sq); a.sk = to_s(sk); a.sv = to_s(sv); a.so = to_s(so);
+  a.B = B; a.N = N; a.H = H; a.d = d;
+  a.scale = resolve_scale(softmax_scale, d);
+  a.wl = window_left;
+  a.wr = window_right;
+  normalise_window(causal, &a.wl, &a.wr);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  int dev;
+  DeviceInfo di;
+  FA2_TRY(current_device(&dev, &di));
+
+  if (dtype == FA2_F32) {
+    dim3 grid((N + 3) / 4, H, B);
+    if (d == 64) simt_fwd_kernel<float, 64><<<grid, 128, 0, st>>>(a);
+    else simt_fwd_kernel<float, 128><<<grid, 128, 0, st>>>(a);
+    return launched(1);
+  }
+  if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;  // sm_100a kernels only
+  const int heavy_first = (a.wr >= 0 || a.wl >= 0) ? 1 : 0;
+  if (d == 128) {
+    return alibi_slopes ? launch_fwd_sm100<128, true>(a, sq, sk, sv, so, dev, heavy_first, st, g_smem_fwd128a)
+                        : launch_fwd_sm100<128, false>(a, sq, sk, sv, so, dev, heavy_first, st, g_smem_fwd128);
+  }
+  return alibi_slopes ? launch_fwd_sm100<64, true>(a, sq, sk, sv, so, dev, heavy_first, st, g_smem_fwd64a)
+                      : launch_fwd_sm100<64, false>(a, sq, sk, sv, so, dev, heavy_first, st, g_smem_fwd64);
+}
+
+fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D, int B, int N, int H, int d,
+                              fa2_dtype dtype, fa2_strides so, fa2_strides sdo, void* stream) {
+  FA2_TRY(check_shape(B, N, H, d, dtype));
+  FA2_TRY(check_tensor(o, so, dtype));
+  FA2_TRY(check_tensor(dout, sdo, dtype));
+  if (D == nullptr || !aligned16(D)) return FA2_ERR_INVALID_ARG;
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.o = const_cast<void*>(o); a.dout = dout; a.dvec = D;
+  a.so = to_s(so); a.sdo = to_s(sdo);
+  a.B = B; a.N = N; a.H = H; a.d = d;
+  int dev;
+  DeviceInfo di;
+  FA2_TRY(current_device(&dev, &di));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long rows = (long long)B * H * N;
+  const int lanes = dtype == FA2_BF16 ? d / 8 : d / 4;
+  const long long per_block = 256 / lanes;
+  const unsigned grid = unsigned((rows + per_block - 1) / per_block);
+  if (dtype == FA2_BF16) {
+    if (d == 64) bwd_preprocess_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(a);
+    else bwd_preprocess_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(a);
+  } else {
+    if (d == 64) bwd_preprocess_kernel<float, 64><<<grid, 256, 0, st>>>(a);
+    else bwd_preprocess_kernel<float, 128><<<grid, 256, 0, st>>>(a);
+  }
+  return launched(1);
+}
+
+size_t fa2_bwd_workspace_size(int B, int N, int H, int d, fa2_dtype dtype, int deterministic) {
+  if (check_shape(B, N, H, d, dtype) != FA2_OK) return 0;
+  if (dtype != FA2_BF16 || deterministic) return 0;
+  const size_t bytes = size_t(B) * H * N * d * sizeof(float);
+  return (bytes + 255) & ~size_t(255);
+}
+
+fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                   const float* D, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, int B, int N, int H, int d, fa2_dtype dtype,
+                   fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides sdo,
+                   fa2_strides sdq, fa2_strides sdk, fa2_strides sdv, float softmax_scale,
+                   int causal, int window_left, int window_right, const float* alibi_slopes,
+                   float dropout_p, int deterministic, void* stream) {
+  FA2_TRY(check_shape(B, N, H, d, dtype));
+  FA2_TRY(check_tensor(q, sq, dtype));
+  FA2_TRY(check_tensor(k, sk, dtype));
+  FA2_TRY(check_tensor(v, sv, dtype));
+  FA2_TRY(check_tensor(dout, sdo, dtype));
+  FA2_TRY(check_tensor(dq, sdq, dtype));
+  FA2_TRY(check_tensor(dk, sdk, dtype));
+  FA2_TRY(check_tensor(dv, sdv, dtype));
+  if (lse == nullptr || !aligned16(lse) || D == nullptr || !aligned16(D)) return FA2_ERR_INVALID_ARG;
+  FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
+  const size_t need = fa2_bwd_workspace_size(B, N, H, d, dtype, deterministic);
+  if (need > 0) {
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+        workspace_bytes < need)
+      return FA2_ERR_INVALID_ARG;
+  }
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = const_cast<float*>(lse); a.dvec = D;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.alibi = alibi_slopes;
+  a.dq_accum = static_cast<float*>(workspace);
+  a.sq = to_s(sq); a.sk = to_s(sk); a.sv = to_s(sv); a.sdo = to_s(sdo);
+  a.sdq = to_s(sdq); a.sdk = to_s(sdk); a.sdv = to_s(sdv);
+  a.B = B; a.N = N; a.H = H; a.d = d;
+  a.scale = resolve_scale(softmax_scale, d);
+  a.wl = window_left;
+  a.wr = window_right;
+  normalise_window(causal, &a.wl, &a.wr);
+  int dev;
+  DeviceInfo di;
+  FA2_TRY(current_device(&dev, &di));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid((N + 3) / 4, H, B);
+  if (dtype == FA2_F32) {
+    if (d == 64) {
+      simt_bwd_dkdv_kernel<float, 64><<<grid, 128, 0, st>>>(a);
+      simt_bwd_dq_kernel<float, 64><<<grid, 128, 0, st>>>(a);
+    } else {
+      simt_bwd_dkdv_kernel<float, 128><<<grid, 128, 0, st>>>(a);
+      simt_bwd_dq_kernel<float, 128><<<grid, 128, 0, st>>>(a);
+    }
+    return launched(2);
+  }
+  if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;
+  if (d == 128)
+    return alibi_slopes ? launch_bwd_sm100<128, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
+                        : launch_bwd_sm100<128, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
+  return alibi_slopes ? launch_bwd_sm100<64, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
+                      : launch_bwd_sm100<64, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,184 @@
+/*
+ * libfa2 -- exact FlashAttention-2 forward and backward for NVIDIA B200
+ * (sm_100a), behind a plain C ABI.
+ *
+ * What the library computes
+ * -------------------------
+ * For every batch b and head h, with query rows i and key rows j in [0, N):
+ *
+ *     s_ij  = softmax_scale * <q_i, k_j> + bias_ij        (bias: ALiBi, below)
+ *     s_ij  = -inf where the mask hides key j from query i
+ *     P     = softmax over j of s (row by row)
+ *     O     = P V,   LSE_i = log sum_j exp(s_ij)          (natural log)
+ *
+ * This is ordinary (exact) attention: the FlashAttention explainer
+ * "AI基础 | Flash Attention" (yeyulingfeng.com) states in its opening that the
+ * method changes how attention is computed on the GPU, not its result, and
+ * the FlashAttention-2 abstract (arXiv 2307.08691) says "without
+ * approximation".  The N x N score matrix is never written to device memory:
+ * the forward pass streams key/value tiles through on-chip memory with an
+ * online softmax (explainer, "Tiling" and "Online softmax" sections) and
+ * keeps only the per-row log-sum-exp; the backward pass recomputes the
+ * probabilities from Q, K and that statistic (explainer, "Backward pass").
+ *
+ * The options follow the call printed in the "FlashAttention v2" article
+ * (wmrh.cn), §5.1 (API): dropout_p, softmax_scale, causal, window_size =
+ * (left, right), alibi_slopes and deterministic.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors q, k, v, o, dout, dq, dk, dv are [B, N, H, d] with the d index
+ *    contiguous (stride 1) and the other strides given in ELEMENTS by an
+ *    fa2_strides value; every stride must be a multiple of 8 elements
+ *    (16 bytes) for bf16 and of 4 elements for fp32, and every base pointer
+ *    16-byte aligned.  lse and D are dense fp32 [B, H, N].
+ *  - All pointers are DEVICE pointers, owned by the caller; the library
+ *    allocates no device memory and keeps no state between calls except a
+ *    small cache of device properties and the device status word read by
+ *    fa2_device_status().
+ *  - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *    default stream); nothing is synchronised.
+ *  - Every argument is checked before anything is launched.  An invalid
+ *    argument returns FA2_ERR_INVALID_ARG and launches nothing; a valid but
+ *    unimplemented combination returns FA2_ERR_UNSUPPORTED; a CUDA error at
+ *    launch returns FA2_ERR_CUDA.
+ *  - Supported shapes: d in {64, 128}; 1 <= N; B, H >= 1; the key/value
+ *    sequence has the same length and head count as the queries.
+ *  - dtype FA2_BF16: bf16 inputs/outputs, fp32 accumulation on the tensor
+ *    cores.  dtype FA2_F32: fp32 inputs/outputs with full fp32 arithmetic
+ *    (CUDA cores), for checks at 1e-4.
+ */
+#ifndef FA2_H_
+#define FA2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA2_BF16 = 0,
+  FA2_F32 = 1
+} fa2_dtype;
+
+typedef enum {
+  FA2_OK = 0,
+  FA2_ERR_INVALID_ARG = 1,     /* a pointer, shape, stride or option is invalid */
+  FA2_ERR_UNSUPPORTED = 2,     /* valid, but not implemented (e.g. dropout_p != 0) */
+  FA2_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed */
+  FA2_ERR_DEVICE_TIMEOUT = 4   /* a kernel gave up a bounded wait (see fa2_device_status) */
+} fa2_status;
+
+/* Element strides of a [B, N, H, d] tensor; the d stride is always 1. */
+typedef struct {
+  int64_t b;
+  int64_t n;
+  int64_t h;
+} fa2_strides;
+
+/*
+ * Forward pass: O = softmax(scale * Q K^T + bias, masked) V and the per-row
+ * natural-log log-sum-exp.
+ *
+ *   q, k, v       [B, N, H, d] inputs (dtype), strides sq, sk, sv.
+ *   o             [B, N, H, d] output (dtype), strides so.  May not alias q/k/v.
+ *   lse           [B, H, N] fp32 output, dense.
+ *   softmax_scale <= 0 selects 1/sqrt(d) (the "softmax_scale=None" default).
+ *   causal        nonzero: key j is visible to query i only if j <= i
+ *                 (equivalent to window_right = 0).
+ *   window_left, window_right
+ *                 sliding window: key j is visible to query i only if
+ *                 i - window_left <= j <= i + window_right (inclusive);
+ *                 a negative value means unbounded on that side
+ *                 ("window_size=(-1,-1)" is the default).
+ *   alibi_slopes  NULL, or a device fp32 [H] array; adds -slope_h * |i - j|
+ *                 to the scaled score (linear-bias attention).
+ *   dropout_p     must be 0 (anything else returns FA2_ERR_UNSUPPORTED).
+ *
+ * A query row that sees no key (impossible with the masks above, since the
+ * diagonal is always visible) gets O = 0 and lse = -inf.  The result is
+ * bitwise identical between runs with the same inputs and shapes.
+ */
+fa2_status fa2_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int N, int H, int d, fa2_dtype dtype,
+                   fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides so,
+                   float softmax_scale, int causal, int window_left, int window_right,
+                   const float* alibi_slopes, float dropout_p, void* stream);
+
+/*
+ * Backward pre-processing: D[b, h, i] = sum_c dO[b, i, h, c] * O[b, i, h, c]
+ * in fp32 (the row sums of dO o O that the softmax gradient needs).
+ *
+ *   o, dout  [B, N, H, d] (dtype), strides so, sdo.
+ *   D        [B, H, N] fp32 output, dense.
+ */
+fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D,
+                              int B, int N, int H, int d, fa2_dtype dtype,
+                              fa2_strides so, fa2_strides sdo, void* stream);
+
+/*
+ * Bytes of device workspace fa2_bwd needs for these shapes (an fp32 dQ
+ * accumulator for bf16, nothing for fp32).  The caller allocates it; its
+ * contents on entry do not matter.  Returns 0 for invalid shapes.
+ */
+size_t fa2_bwd_workspace_size(int B, int N, int H, int d, fa2_dtype dtype, int deterministic);
+
+/*
+ * Backward pass: dQ, dK, dV of L = sum(O o dO) given the forward's lse and
+ * the pre-processed D.  The probabilities are recomputed from q, k and lse.
+ *
+ *   q, k, v, dout    [B, N, H, d] inputs (dtype) with strides sq, sk, sv, sdo.
+ *   lse, D           [B, H, N] fp32 from fa2_fwd and fa2_bwd_preprocess.
+ *   dq, dk, dv       [B, N, H, d] outputs (dtype) with strides sdq, sdk, sdv.
+ *   workspace        device buffer of at least workspace_bytes >=
+ *                    fa2_bwd_workspace_size(...) bytes, 256-byte aligned.
+ *   softmax_scale, causal, window_left, window_right, alibi_slopes, dropout_p
+ *                    exactly as passed to fa2_fwd.
+ *   deterministic    0: dQ partial sums from different key blocks are added
+ *                    with fp32 atomics (fast, order not fixed);
+ *                    nonzero: dQ is produced by an ordered pass with no
+ *                    atomics, so dq, dk and dv are bitwise repeatable.
+ */
+fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout,
+                   const float* lse, const float* D, void* dq, void* dk, void* dv,
+                   void* workspace, size_t workspace_bytes,
+                   int B, int N, int H, int d, fa2_dtype dtype,
+                   fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides sdo,
+                   fa2_strides sdq, fa2_strides sdk, fa2_strides sdv,
+                   float softmax_scale, int causal, int window_left, int window_right,
+                   const float* alibi_slopes, float dropout_p, int deterministic,
+                   void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* fa2_strerror(fa2_status status);
+
+/*
+ * Reads (and, if `clear` is nonzero, resets) the device status word of the
+ * current device.  Synchronises the device.  *code receives 0 if no kernel
+ * has given up a bounded wait since the last clear, else the code of the
+ * first wait that did.  Returns FA2_ERR_DEVICE_TIMEOUT when *code != 0,
+ * FA2_OK otherwise, FA2_ERR_CUDA on a CUDA error.
+ */
+fa2_status fa2_device_status(int* code, int clear);
+
+/*
+ * Sets the time limit, in milliseconds, of every bounded wait inside the
+ * kernels launched afterwards by this process (default 1000 ms).  Values
+ * < 1 are rejected with FA2_ERR_INVALID_ARG.
+ */
+fa2_status fa2_set_wait_limit_ms(int ms);
+
+/*
+ * Number of kernels this library has launched in this process since it was
+ * loaded (all devices, all entry points).  Lets a caller count the device
+ * work of a region: read it before and after.
+ */
+uint64_t fa2_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA2_H_ */

@@ -1,0 +1,108 @@
+"""The C ABI without a GPU: the library loads, exports every symbol its
+header declares, and rejects invalid arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from exact_attention_147_b200 import build as fa2_build
+from exact_attention_147_b200 import fa2 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa2.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa2_build.build()
+    return F.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa2_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(F.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_strerror(lib):
+    for code in range(5):
+        assert F.strerror(code).startswith("FA2_")
+    assert "unknown" in F.strerror(99)
+
+
+# Fake, 16-byte aligned device addresses: every call below fails its argument
+# checks, so nothing dereferences them.
+P = ctypes.c_void_p(0x100000)
+S128 = F.Strides(8 * 2048 * 16 * 128 // 8, 16 * 128, 128)   # [B,N,H,d] dense strides
+
+
+def call_fwd(lib, **kw):
+    a = dict(q=P, k=P, v=P, o=ctypes.c_void_p(0x200000), lse=P, B=1, N=256, H=2, d=128,
+             dtype=F.FA2_BF16, s=S128, scale=0.0, causal=0, wl=-1, wr=-1, alibi=None,
+             dropout=0.0)
+    a.update(kw)
+    return lib.fa2_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["N"], a["H"], a["d"],
+                       a["dtype"], a["s"], a["s"], a["s"], a["s"], a["scale"], a["causal"],
+                       a["wl"], a["wr"], a["alibi"], a["dropout"], None)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(q=None), dict(k=None), dict(lse=None), dict(d=96), dict(d=0), dict(N=0), dict(B=0),
+    dict(H=-1), dict(dtype=7), dict(q=ctypes.c_void_p(0x100008)),
+    dict(s=F.Strides(8, 12, 128)), dict(s=F.Strides(0, 128, 128)), dict(scale=float("nan")),
+    dict(dropout=float("nan")), dict(dropout=1.5), dict(alibi=ctypes.c_void_p(0x100002)),
+    dict(o=P),  # output aliases an input
+])
+def test_fwd_rejects_invalid(lib, bad):
+    assert call_fwd(lib, **bad) == F.FA2_ERR_INVALID_ARG
+
+
+def test_fwd_dropout_unsupported(lib):
+    assert call_fwd(lib, dropout=0.1) == F.FA2_ERR_UNSUPPORTED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_valid_call_without_device_is_cuda_error(lib):
+    assert call_fwd(lib) == F.FA2_ERR_CUDA
+
+
+def test_preprocess_and_bwd_reject_invalid(lib):
+    s = S128
+    assert lib.fa2_bwd_preprocess(P, P, None, 1, 256, 2, 128, F.FA2_BF16, s, s, None) == \
+        F.FA2_ERR_INVALID_ARG
+    assert lib.fa2_bwd_preprocess(P, P, P, 1, 256, 2, 100, F.FA2_BF16, s, s, None) == \
+        F.FA2_ERR_INVALID_ARG
+    need = lib.fa2_bwd_workspace_size(1, 256, 2, 128, F.FA2_BF16, 0)
+    # workspace too small
+    st = lib.fa2_bwd(P, P, P, P, P, P, ctypes.c_void_p(0x300000), ctypes.c_void_p(0x400000),
+                     ctypes.c_void_p(0x500000), ctypes.c_void_p(0x600000), need - 1,
+                     1, 256, 2, 128, F.FA2_BF16, s, s, s, s, s, s, s, 0.0, 0, -1, -1, None,
+                     0.0, 0, None)
+    assert st == F.FA2_ERR_INVALID_ARG
+    # dropout
+    st = lib.fa2_bwd(P, P, P, P, P, P, ctypes.c_void_p(0x300000), ctypes.c_void_p(0x400000),
+                     ctypes.c_void_p(0x500000), ctypes.c_void_p(0x600000), need,
+                     1, 256, 2, 128, F.FA2_BF16, s, s, s, s, s, s, s, 0.0, 0, -1, -1, None,
+                     0.2, 0, None)
+    assert st == F.FA2_ERR_UNSUPPORTED
+
+
+def test_workspace_size(lib):
+    assert lib.fa2_bwd_workspace_size(2, 300, 3, 64, F.FA2_BF16, 0) == 2 * 300 * 3 * 64 * 4
+    assert lib.fa2_bwd_workspace_size(1, 256, 2, 64, F.FA2_F32, 0) == 0
+    assert lib.fa2_bwd_workspace_size(1, 256, 2, 96, F.FA2_BF16, 0) == 0
+
+
+def test_wait_limit(lib):
+    assert lib.fa2_set_wait_limit_ms(0) == F.FA2_ERR_INVALID_ARG
+    assert lib.fa2_set_wait_limit_ms(1000) == F.FA2_OK
