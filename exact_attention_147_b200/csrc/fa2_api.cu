@@ -254,6 +254,8 @@ const char* fa2_strerror(fa2_status s) {
     case FA2_ERR_UNSUPPORTED: return "FA2_ERR_UNSUPPORTED: valid but not implemented";
     case FA2_ERR_CUDA: return "FA2_ERR_CUDA: a CUDA call failed";
     case FA2_ERR_DEVICE_TIMEOUT: return "FA2_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait";
+    case FA2_ERR_SCRATCH_LIMIT:
+      return "FA2_ERR_SCRATCH_LIMIT: B*H*N*d exceeds the fixed scratch of fa2_bwd_noalloc";
   }
   return "unknown fa2_status";
 }
@@ -415,6 +417,80 @@ fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout
                         : launch_bwd_sm100<128, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
   return alibi_slopes ? launch_bwd_sm100<64, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
                       : launch_bwd_sm100<64, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
+}
+
+// ---------------------------------------------------------------------------
+// fa2_bwd_noalloc: fa2_bwd (bf16, non-deterministic) with its fp32 dQ
+// accumulator in a fixed device array instead of caller workspace.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+// The scratch array.  In host code this name is only a stand-in for the
+// device object: its device address comes from cudaGetSymbolAddress, looked
+// up once per device with that device current.
+static __device__ __align__(256) float g_fa2_noalloc_dq[FA2_NOALLOC_MAX_DQ_FLOATS];
+float* g_noalloc_addr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+fa2_status noalloc_scratch(int dev, float** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_fa2_noalloc_dq) != cudaSuccess || ptr == nullptr)
+      return FA2_ERR_CUDA;
+    g_noalloc_addr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_noalloc_addr[dev];
+  return FA2_OK;
+}
+}  // namespace
+
+extern "C" {
+
+fa2_status fa2_bwd_noalloc(const void* q, const void* k, const void* v, const void* dout,
+                           const float* lse, const float* D, void* dq, void* dk, void* dv, int B,
+                           int N, int H, int d, fa2_strides sq, fa2_strides sk, fa2_strides sv,
+                           fa2_strides sdo, fa2_strides sdq, fa2_strides sdk, fa2_strides sdv,
+                           float softmax_scale, int causal, int window_left, int window_right,
+                           const float* alibi_slopes, float dropout_p, void* stream) {
+  const fa2_dtype dtype = FA2_BF16;
+  FA2_TRY(check_shape(B, N, H, d, dtype));
+  FA2_TRY(check_tensor(q, sq, dtype));
+  FA2_TRY(check_tensor(k, sk, dtype));
+  FA2_TRY(check_tensor(v, sv, dtype));
+  FA2_TRY(check_tensor(dout, sdo, dtype));
+  FA2_TRY(check_tensor(dq, sdq, dtype));
+  FA2_TRY(check_tensor(dk, sdk, dtype));
+  FA2_TRY(check_tensor(dv, sdv, dtype));
+  if (lse == nullptr || !aligned16(lse) || D == nullptr || !aligned16(D)) return FA2_ERR_INVALID_ARG;
+  FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
+  if ((unsigned long long)B * H * N * d > (unsigned long long)FA2_NOALLOC_MAX_DQ_FLOATS)
+    return FA2_ERR_SCRATCH_LIMIT;
+  int dev;
+  DeviceInfo di;
+  FA2_TRY(current_device(&dev, &di));
+  if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;
+  float* scratch = nullptr;
+  FA2_TRY(noalloc_scratch(dev, &scratch));
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = const_cast<float*>(lse); a.dvec = D;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.alibi = alibi_slopes;
+  a.dq_accum = scratch;  // cleared by the first kernel of the launch sequence
+  a.sq = to_s(sq); a.sk = to_s(sk); a.sv = to_s(sv); a.sdo = to_s(sdo);
+  a.sdq = to_s(sdq); a.sdk = to_s(sdk); a.sdv = to_s(sdv);
+  a.B = B; a.N = N; a.H = H; a.d = d;
+  a.scale = resolve_scale(softmax_scale, d);
+  a.wl = window_left;
+  a.wr = window_right;
+  normalise_window(causal, &a.wl, &a.wr);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return alibi_slopes ? launch_bwd_sm100<128, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st)
+                        : launch_bwd_sm100<128, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st);
+  return alibi_slopes ? launch_bwd_sm100<64, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st)
+                      : launch_bwd_sm100<64, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st);
 }
 
 }  // extern "C"

@@ -32,11 +32,13 @@ FA2_ERR_INVALID_ARG = 1
 FA2_ERR_UNSUPPORTED = 2
 FA2_ERR_CUDA = 3
 FA2_ERR_DEVICE_TIMEOUT = 4
+FA2_ERR_SCRATCH_LIMIT = 5
+NOALLOC_MAX_DQ_FLOATS = 4 * 1024 * 1024
 
 # Every symbol include/fa2.h declares.
 EXPORTED = ("fa2_fwd", "fa2_bwd_preprocess", "fa2_bwd_workspace_size", "fa2_bwd",
             "fa2_strerror", "fa2_device_status", "fa2_set_wait_limit_ms",
-            "fa2_kernel_launches")
+            "fa2_kernel_launches", "fa2_bwd_noalloc")
 
 
 class Strides(ctypes.Structure):
@@ -78,6 +80,9 @@ def load_library(path: str = LIB_PATH):
     lib.fa2_device_status.restype = i
     lib.fa2_set_wait_limit_ms.argtypes = [i]
     lib.fa2_set_wait_limit_ms.restype = i
+    lib.fa2_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
+                                    s, s, s, s, s, s, s, f, i, i, i, vp, f, vp]
+    lib.fa2_bwd_noalloc.restype = i
     lib.fa2_kernel_launches.argtypes = []
     lib.fa2_kernel_launches.restype = ctypes.c_uint64
     _lib = lib

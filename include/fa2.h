@@ -68,7 +68,8 @@ typedef enum {
   FA2_ERR_INVALID_ARG = 1,     /* a pointer, shape, stride or option is invalid */
   FA2_ERR_UNSUPPORTED = 2,     /* valid, but not implemented (e.g. dropout_p != 0) */
   FA2_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed */
-  FA2_ERR_DEVICE_TIMEOUT = 4   /* a kernel gave up a bounded wait (see fa2_device_status) */
+  FA2_ERR_DEVICE_TIMEOUT = 4,  /* a kernel gave up a bounded wait (see fa2_device_status) */
+  FA2_ERR_SCRATCH_LIMIT = 5    /* problem too large for fa2_bwd_noalloc's fixed scratch */
 } fa2_status;
 
 /* Element strides of a [B, N, H, d] tensor; the d stride is always 1. */
@@ -150,6 +151,46 @@ fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout
                    float softmax_scale, int causal, int window_left, int window_right,
                    const float* alibi_slopes, float dropout_p, int deterministic,
                    void* stream);
+
+/*
+ * fa2_bwd_noalloc: the bf16 backward pass without any caller-provided or
+ * library-allocated workspace.  (No counterpart in the paper: this is an
+ * interface convenience, not part of the method.)
+ *
+ * Some callers cannot allocate device memory at the point where they run
+ * the backward pass: code inside a host framework that owns every byte of
+ * device memory through its own pool and forbids cudaMalloc after start-up,
+ * plugin interfaces that hand over inputs and outputs but no workspace, and
+ * latency-critical loops where an allocation may block on the driver.  For
+ * them this entry point takes the fp32 dQ accumulator from a fixed array
+ * compiled into the library (FA2_NOALLOC_MAX_DQ_FLOATS floats, 16 MiB,
+ * present on every GPU that loads the library until the process exits).
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments and results are those of fa2_bwd with dtype FA2_BF16 and
+ * deterministic = 0 (dQ partial sums added with fp32 atomics).  The caller
+ * still provides q, k, v, dout, lse, D, dq, dk and dv.
+ *
+ *   Limit:   B * H * N * d must not exceed FA2_NOALLOC_MAX_DQ_FLOATS;
+ *            larger problems return FA2_ERR_SCRATCH_LIMIT and launch
+ *            nothing (use fa2_bwd with a workspace instead).
+ *   Set-up:  the first call on a device looks up the device address of the
+ *            array (cudaGetSymbolAddress) with that device current; make
+ *            that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array.  The accumulator
+ *            is cleared at the start of each call, but two calls whose
+ *            kernels overlap on the GPU (different streams, no ordering
+ *            between them) race on it and give wrong gradients; order such
+ *            calls on one stream or with events.
+ */
+#define FA2_NOALLOC_MAX_DQ_FLOATS (4u * 1024u * 1024u)
+fa2_status fa2_bwd_noalloc(const void* q, const void* k, const void* v, const void* dout,
+                           const float* lse, const float* D, void* dq, void* dk, void* dv,
+                           int B, int N, int H, int d,
+                           fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides sdo,
+                           fa2_strides sdq, fa2_strides sdk, fa2_strides sdv,
+                           float softmax_scale, int causal, int window_left, int window_right,
+                           const float* alibi_slopes, float dropout_p, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* fa2_strerror(fa2_status status);
