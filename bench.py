@@ -52,6 +52,35 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+# ------------------------------------------------------------------ traffic
+KERNEL_SOURCES = {
+    "fa2_fwd": ["sm100_ptx.cuh", "attn_common.cuh", "fwd_sm100.cuh"],
+    "fa2_bwd": ["sm100_ptx.cuh", "attn_common.cuh", "bwd_sm100.cuh", "fwd_sm100.cuh"],
+}
+
+
+def sources_hash(call):
+    import hashlib
+    m = hashlib.sha256()
+    for f in sorted(KERNEL_SOURCES[call]):
+        with open(os.path.join(ROOT, "exact_attention_147_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    return m.hexdigest()[:16]
+
+
+def captured_traffic(call):
+    """DRAM bytes per launch from the committed ncu capture, or None when the
+    kernel sources changed since that capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+            t = json.load(fh).get(call)
+        if t and t.get("sources_sha256") == sources_hash(call):
+            return t["bytes"]
+    except Exception:
+        pass
+    return None
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clock/throttle sampling during the timed region."""
@@ -326,13 +355,7 @@ def run_gpu(args):
     pre_gbs = pre_bytes / (ms_pre * 1e-3) / 1e9
     dominant = "fa2_bwd" if ms_bwd >= ms_fwd else "fa2_fwd"
     achieved = bwd_tflops if dominant == "fa2_bwd" else fwd_tflops
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            traffic = json.load(open(tpath)).get(dominant)
-        except Exception:
-            traffic = None
+    traffic = captured_traffic(dominant)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
                 "frac": achieved / sustained, "traffic": traffic, "kernel": dominant,
                 "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a "
