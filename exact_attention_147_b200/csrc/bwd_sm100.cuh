@@ -46,6 +46,7 @@ namespace fa2 {
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;   // inputs, box {64,1,128,1}
   CUtensorMap tm_dq, tm_dk, tm_dv;       // outputs (bf16), same boxes
+  CUtensorMap tm_dqacc;                  // fp32 [B*H, N, d] accumulator, box {32,128,1}
   const float* lse;                      // [B,H,N]
   const float* dvec;                     // [B,H,N]
   float* dq_accum;                       // [B,H,N,d] fp32 (kernel 1 with dQ)
@@ -74,10 +75,14 @@ struct BwdCfg {
   static constexpr int OFF_SIDE = OFF_DS + DS_BYTES;
   static constexpr int OFF_BARS = OFF_SIDE + Q_STAGES * SIDE_BYTES;
   // kv_full, Q full/empty, dO full/empty, s_full, dp_full, p_ready, ds_ready,
-  // dq_full, dq_free, acc_full, drain
-  static constexpr int NBARS = 1 + 2 * Q_STAGES + 2 * DO_STAGES + 8;
+  // dq_full, dq_free, acc_full, stage_free, drain
+  static constexpr int NBARS = 1 + 2 * Q_STAGES + 2 * DO_STAGES + 9;
   static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16 + 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 512;
+  // registers per thread after the warpgroup re-balancing (see kernel 1)
+  static constexpr int REGS_COMPUTE = 176, REGS_DRAIN = 96, REGS_MISC = 64;
+  static constexpr int REGS_AT_LAUNCH = (2 * 128 * REGS_COMPUTE + 128 * REGS_DRAIN + 128 * REGS_MISC) / 512;
+  static_assert(REGS_AT_LAUNCH == 128, "register split must use exactly the launch budget");
 };
 
 template <int HD>
@@ -120,9 +125,22 @@ __device__ __forceinline__ void st_sw128_row32(uint8_t* tile, int row, int col0,
 
 // ---------------------------------------------------------------------------
 // Kernel 1: dK, dV (and the atomically accumulated dQ when WITH_DQ)
+//
+// 16 warps: warpgroups 0 and 1 compute (thread = key row; warpgroup w owns
+// query columns [64w, 64w+64) of every S^T / dP^T tile), warpgroup 2 drains
+// dQ (thread = query row), warp 12 loads, warp 13 issues the MMAs.  Register
+// budget after the split: compute 176, drain 96, loader/MMA warpgroup 64
+// (2*128*176 + 128*96 + 128*64 = 65536 = 512 threads x 128 at launch; the
+// host checks the launch register count before every launch).
+//
+// dQ path: the drain warpgroup reads the dQ tile out of TMEM 64 columns at
+// a time, stages each round in the dS^T tile of shared memory (free once the
+// dQ MMA is done) and adds it into the fp32 accumulator with TMA bulk
+// reductions, which go through the TMA unit rather than the load/store
+// queues.  TMEM is released after the last round is read.
 // ---------------------------------------------------------------------------
 template <int HD, bool ALIBI, bool WITH_DQ>
-__global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<HD>;
   using namespace bwd_detail;
   constexpr int QS = C::Q_STAGES, DS = C::DO_STAGES;
@@ -148,12 +166,14 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   const uint32_t s_full = b0 + 8u * (1 + 2 * QS + 2 * DS);
   const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24;
   const uint32_t dq_full = s_full + 32, dq_free = s_full + 40, acc_full = s_full + 48;
+  const uint32_t stage_free = s_full + 56;
   const uint32_t drain_bar = b0 + 8u * (C::NBARS - 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   AbortFlag ab{abort_flag};
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int wg = warp / 4;
   const int nhb = p.H * p.B;
   int kb, hb;
   if (p.heavy_first) {  // causal: key block 0 is seen by the most query blocks
@@ -176,11 +196,14 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
     *abort_flag = 0;
     for (int i = 0; i < C::NBARS; ++i) {
       const uint32_t bar = b0 + 8u * i;
-      bar_init(bar, (bar == p_ready || bar == ds_ready || bar == dq_free) ? 128 : 1);
+      uint32_t cnt = 1;
+      if (bar == p_ready || bar == ds_ready) cnt = 256;
+      if (bar == dq_free) cnt = 128;
+      bar_init(bar, cnt);
     }
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -189,67 +212,74 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      bar_arrive_expect_tx(kv_full, 2 * C::TILE);
-      for (int c = 0; c < NCH; ++c) {
-        tma_load_4d(smem_u32(sK + c * 16384), &p.tm_k, kv_full, c * 64, h, k0, b);
-        tma_load_4d(smem_u32(sV + c * 16384), &p.tm_v, kv_full, c * 64, h, k0, b);
-      }
-    }
-    int issued_q = 0, issued_do = 0;
-    bool ok = true;
-    for (int it = 0; it < nq && ok; ++it) {
-      const int i0 = (qb_begin + it) * 128;
-      const int sq = it % QS;
-      ok = wait_bar(q_empty(sq), ((it / QS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 0);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      // log2-scaled LSE and D of this query block, +inf / 0 past N
-      float* side = sSide + sq * 256;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = lane + 32 * e;
-        const int i = i0 + c;
-        float l2 = CUDART_INF_F, dv = 0.f;
-        if (i < p.N) {
-          const float l = p.lse[head_off + i];
-          l2 = l == -CUDART_INF_F ? CUDART_INF_F : l * LOG2E;
-          dv = p.dvec[head_off + i];
+  if (wg == 3) {
+    regs_dec<C::REGS_MISC>();
+    if (warp == 12) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0) {
+        bar_arrive_expect_tx(kv_full, 2 * C::TILE);
+        for (int c = 0; c < NCH; ++c) {
+          tma_load_4d(smem_u32(sK + c * 16384), &p.tm_k, kv_full, c * 64, h, k0, b);
+          tma_load_4d(smem_u32(sV + c * 16384), &p.tm_v, kv_full, c * 64, h, k0, b);
         }
-        side[c] = l2;
-        side[128 + c] = dv;
       }
-      __threadfence_block();
-      __syncwarp();
+      int issued_q = 0, issued_do = 0;
+      bool ok = true;
+      for (int it = 0; it < nq && ok; ++it) {
+        const int i0 = (qb_begin + it) * 128;
+        const int sq = it % QS;
+        // log2-scaled LSE and D of this query block, +inf / 0 past N; loaded
+        // before waiting for the slot so the latency overlaps the wait
+        float l2v[4], dvv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = i0 + lane + 32 * e;
+          l2v[e] = CUDART_INF_F;
+          dvv[e] = 0.f;
+          if (i < p.N) {
+            const float l = p.lse[head_off + i];
+            l2v[e] = l == -CUDART_INF_F ? CUDART_INF_F : l * LOG2E;
+            dvv[e] = p.dvec[head_off + i];
+          }
+        }
+        ok = wait_bar(q_empty(sq), ((it / QS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 0);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        float* side = sSide + sq * 256;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          side[lane + 32 * e] = l2v[e];
+          side[128 + lane + 32 * e] = dvv[e];
+        }
+        __threadfence_block();
+        __syncwarp();
+        if (lane == 0) {
+          bar_arrive_expect_tx(q_full(sq), C::TILE);
+          for (int c = 0; c < NCH; ++c)
+            tma_load_4d(smem_u32(sQ + sq * C::TILE + c * 16384), &p.tm_q, q_full(sq), c * 64, h, i0, b);
+        }
+        ++issued_q;
+        const int sd = it % DS;
+        ok = wait_bar(do_empty(sd), ((it / DS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (lane == 0) {
+          bar_arrive_expect_tx(do_full(sd), C::TILE);
+          for (int c = 0; c < NCH; ++c)
+            tma_load_4d(smem_u32(sDO + sd * C::TILE + c * 16384), &p.tm_do, do_full(sd), c * 64, h, i0,
+                        b);
+        }
+        ++issued_do;
+      }
       if (lane == 0) {
-        bar_arrive_expect_tx(q_full(sq), C::TILE);
-        for (int c = 0; c < NCH; ++c)
-          tma_load_4d(smem_u32(sQ + sq * C::TILE + c * 16384), &p.tm_q, q_full(sq), c * 64, h, i0, b);
+        drain_wait(kv_full, 0, p.wait_ns);
+        for (int k = max(0, issued_q - QS); k < issued_q; ++k)
+          drain_wait(q_full(k % QS), (k / QS) & 1, p.wait_ns);
+        for (int k = max(0, issued_do - DS); k < issued_do; ++k)
+          drain_wait(do_full(k % DS), (k / DS) & 1, p.wait_ns);
       }
-      ++issued_q;
-      const int sd = it % DS;
-      ok = wait_bar(do_empty(sd), ((it / DS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 1);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      if (lane == 0) {
-        bar_arrive_expect_tx(do_full(sd), C::TILE);
-        for (int c = 0; c < NCH; ++c)
-          tma_load_4d(smem_u32(sDO + sd * C::TILE + c * 16384), &p.tm_do, do_full(sd), c * 64, h, i0,
-                      b);
-      }
-      ++issued_do;
-    }
-    if (lane == 0) {
-      drain_wait(kv_full, 0, p.wait_ns);
-      for (int k = max(0, issued_q - QS); k < issued_q; ++k) drain_wait(q_full(k % QS), (k / QS) & 1, p.wait_ns);
-      for (int k = max(0, issued_do - DS); k < issued_do; ++k)
-        drain_wait(do_full(k % DS), (k / DS) & 1, p.wait_ns);
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 13 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       const uint32_t id_kq = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       const uint32_t id_pd = idesc_bf16_f32(128, HD, 0, 1);   // dV, dK (B MN-major)
       const uint32_t id_dq = idesc_bf16_f32(128, HD, 1, 1);   // dQ (A and B MN-major)
@@ -261,12 +291,14 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           umma_ss(d_tmem, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024), id_kq, kk > 0);
         }
       };
+      // A operand from TMEM: 16 queries per MMA; queries [64w, 64w+64) were
+      // packed by compute warpgroup w into columns [64w, 64w+32) of its region.
       auto from_tmem = [&](uint32_t d_tmem, uint32_t a_tmem, const uint8_t* bm, bool acc) {
         const uint32_t bb = smem_u32(bm);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(bb + kk * 2048, 16384, 1024), id_pd,
-                  (acc || kk > 0) ? 1u : 0u);
+          umma_ts(d_tmem, a_tmem + 64 * (kk / 4) + (kk % 4) * 8,
+                  sdesc_sw128(bb + kk * 2048, 16384, 1024), id_pd, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = wait_bar(kv_full, 0, ab, p.wait_ns, SITE_BMMA + 0);
       if (ok) ok = wait_bar(q_full(0), 0, ab, p.wait_ns, SITE_BMMA + 1);
@@ -281,7 +313,7 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         if (ok && WITH_DQ && it > 0) ok = wait_bar(dq_free, (it - 1) & 1, ab, p.wait_ns, SITE_BMMA + 3);
         if (!ok) break;
         tc_fence_after();
-        kmajor(tmem + T_DP, sV, sDO + sd * C::TILE);                 // dP^T = V dO^T
+        kmajor(tmem + T_DP, sV, sDO + sd * C::TILE);                      // dP^T = V dO^T
         umma_commit(dp_full);
         ok = wait_bar(p_ready, it & 1, ab, p.wait_ns, SITE_BMMA + 4);
         if (!ok) break;
@@ -293,13 +325,13 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           ok = wait_bar(q_full(sn), ((it + 1) / QS) & 1, ab, p.wait_ns, SITE_BMMA + 5);
           if (!ok) break;
           tc_fence_after();
-          kmajor(tmem + T_S, sK, sQ + sn * C::TILE);                // next S^T
+          kmajor(tmem + T_S, sK, sQ + sn * C::TILE);                     // next S^T
           umma_commit(s_full);
         }
         ok = wait_bar(ds_ready, it & 1, ab, p.wait_ns, SITE_BMMA + 6);
         if (!ok) break;
         tc_fence_after();
-        from_tmem(tmem + T_DK, tmem + T_DP, sQ + sq * C::TILE, it > 0);   // dK += dS^T Q
+        from_tmem(tmem + T_DK, tmem + T_DP, sQ + sq * C::TILE, it > 0);  // dK += dS^T Q
         if (WITH_DQ) {
           // dQ_i = dS K: A = dS (queries x keys) read MN-major from the dS^T
           // tile, B = K (keys x d) MN-major.
@@ -316,41 +348,43 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       umma_commit(drain_bar);
       drain_wait(drain_bar, 0, p.wait_ns);
     }
-  } else if (warp < 4) {
+  } else if (wg < 2) {
+    regs_inc<C::REGS_COMPUTE>();
     // ------------------------------------------------------------ compute (key rows)
-    const int r = warp * 32 + lane;
+    const int r = (warp % 4) * 32 + lane;
     const int j = k0 + r;
+    const int cq = 64 * wg;  // this warpgroup's query columns [cq, cq + 64)
     int lo_q = p.wr >= 0 ? max(0, j - p.wr) : 0;
     int hi_q = p.wl >= 0 ? min(p.N - 1, j + p.wl) : p.N - 1;
     if (j >= p.N) {
       lo_q = 1;
       hi_q = 0;
     }
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
     const float C2 = p.scale_log2;
     float slope2 = 0.f;
     if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
     bool ok = true;
     for (int it = 0; it < nq; ++it) {
-      const int i0 = (qb_begin + it) * 128;
-      const float* side = sSide + (it % QS) * 256;
+      const int i0 = (qb_begin + it) * 128 + cq;
+      const float* side = sSide + (it % QS) * 256 + cq;
       ok = wait_bar(s_full, it & 1, ab, p.wait_ns, SITE_BCOMP + 0);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      float pr[128];
+      float pr[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_base + T_S + c * 32, u);
+        tmem_ld32(tmem + lane_base + T_S + cq + c * 32, u);
 #pragma unroll
         for (int e = 0; e < 32; ++e) pr[c * 32 + e] = __uint_as_float(u[e]);
       }
       tmem_ld_wait();
-      const bool full = (i0 >= lo_q) && (i0 + 127 <= hi_q);
+      const bool full = (i0 >= lo_q) && (i0 + 63 <= hi_q);
       const float fj = float(i0 - j);
 #pragma unroll
-      for (int c = 0; c < 128; c += 4) {
+      for (int c = 0; c < 64; c += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(side + c);
         float x0, x1, x2, x3;
         if (ALIBI) {
@@ -371,43 +405,44 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       }
       if (!full) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
+        for (int c = 0; c < 64; ++c) {
           const int i = i0 + c;
           if (i < lo_q || i > hi_q) pr[c] = 0.f;
         }
       }
-      // P^T (bf16) over the first 64 columns of S^T, for dV += P^T dO
+      // P^T (bf16) into columns [cq, cq+32) of the S^T region (already read)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) w[e] = pack_bf16(pr[c * 32 + 2 * e], pr[c * 32 + 2 * e + 1]);
-        tmem_st16(tmem + lane_base + T_S + c * 16, w);
+        tmem_st16(tmem + lane_base + T_S + cq + c * 16, w);
       }
       tmem_st_wait();
       tc_fence_before();
       bar_arrive(p_ready);
       // dS^T = P^T o (dP^T - D), 32 columns at a time
       ok = wait_bar(dp_full, it & 1, ab, p.wait_ns, SITE_BCOMP + 1);
+      // the dS^T tile doubles as the dQ staging buffer of the previous block
+      if (WITH_DQ && it > 0 && ok) ok = wait_bar(stage_free, (it - 1) & 1, ab, p.wait_ns, SITE_BCOMP + 3);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_base + T_DP + c * 32, u);
+        tmem_ld32(tmem + lane_base + T_DP + cq + c * 32, u);
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int cc = c * 32 + 2 * e;
-          const float d0 = pr[cc] * (__uint_as_float(u[2 * e]) - side[128 + cc]);
-          const float d1 = pr[cc + 1] * (__uint_as_float(u[2 * e + 1]) - side[128 + cc + 1]);
-          w[e] = pack_bf16(d0, d1);
+          w[e] = pack_bf16(pr[cc] * (__uint_as_float(u[2 * e]) - side[128 + cc]),
+                           pr[cc + 1] * (__uint_as_float(u[2 * e + 1]) - side[128 + cc + 1]));
         }
-        // columns already read: written below the read position
-        tmem_st16(tmem + lane_base + T_DP + c * 16, w);
-        if (WITH_DQ) st_sw128_row32(sDS, r, c * 32, w);
+        // written over columns this thread has already read
+        tmem_st16(tmem + lane_base + T_DP + cq + c * 16, w);
+        if (WITH_DQ) st_sw128_row32(sDS, r, cq + c * 32, w);
       }
       tmem_st_wait();
       if (WITH_DQ) fence_proxy_async_smem();
@@ -419,26 +454,28 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
     if (ok) {
-      // dV and dK rows -> bf16 -> the V and K tiles (free now) -> TMA store
+      // this warpgroup's half of the d columns of dV and dK -> bf16 -> the
+      // V and K tiles (free now) -> TMA store
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = 0; c < HD / 64; ++c) {
+        const int col = wg * (HD / 2) + c * 32;
         uint32_t u[32], w[16];
-        tmem_ld32(tmem + lane_base + T_DV + c * 32, u);
+        tmem_ld32(tmem + lane_base + T_DV + col, u);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e) w[e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
-        st_sw128_row32(sV, r, c * 32, w);
-        tmem_ld32(tmem + lane_base + T_DK + c * 32, u);
+        st_sw128_row32(sV, r, col, w);
+        tmem_ld32(tmem + lane_base + T_DK + col, u);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16(__uint_as_float(u[2 * e]) * p.scale, __uint_as_float(u[2 * e + 1]) * p.scale);
-        st_sw128_row32(sK, r, c * 32, w);
+        st_sw128_row32(sK, r, col, w);
       }
     }
     fence_proxy_async_smem();
-    named_bar_sync(1, 128);
-    if (ok && r == 0) {
+    named_bar_sync(1, 256);
+    if (ok && threadIdx.x == 0) {
       for (int c = 0; c < NCH; ++c) {
         tma_store_4d(&p.tm_dv, smem_u32(sV + c * 16384), c * 64, h, k0, b);
         tma_store_4d(&p.tm_dk, smem_u32(sK + c * 16384), c * 64, h, k0, b);
@@ -446,38 +483,70 @@ __global__ void __launch_bounds__(320, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       bulk_commit();
       bulk_wait_all();
     }
-  } else if (WITH_DQ && warp < 8) {
-    // ------------------------------------------------------------ dQ drain (query rows)
-    const int q = (warp - 4) * 32 + lane;
-    const uint32_t lane_base = uint32_t((warp - 4) * 32) << 16;
-    for (int it = 0; it < nq; ++it) {
-      const int i = (qb_begin + it) * 128 + q;
-      bool ok = wait_bar(dq_full, it & 1, ab, p.wait_ns, SITE_BRED);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      float acc[HD];
+  } else {
+    regs_dec<C::REGS_DRAIN>();
+    if (WITH_DQ) {
+      // ---------------------------------------------------------- dQ drain (query rows)
+      const int q = (warp % 4) * 32 + lane;
+      const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
+      const int bh = b * p.H + h;
+      for (int it = 0; it < nq; ++it) {
+        const int i0 = (qb_begin + it) * 128;
+        bool ok = wait_bar(dq_full, it & 1, ab, p.wait_ns, SITE_BRED);
+        // leave together: the rounds below use a warpgroup-wide barrier
+        if (!named_bar_all(2, 128, ok)) break;
+        tc_fence_after();
+        // 64 columns per round: read them from TMEM, stage them as two
+        // 32-column (128-byte) swizzled boxes of 128 rows in the dS^T tile,
+        // and add each box into the accumulator with one bulk reduction.
+        // TMEM is released as soon as the last round's columns are read.
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_base + T_DP + c * 32, u);
+        for (int rd = 0; rd < HD / 64; ++rd) {
+          float acc[64];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) acc[c * 32 + e] = __uint_as_float(u[e]);
+          for (int c = 0; c < 2; ++c) {
+            uint32_t u[32];
+            tmem_ld32(tmem + lane_base + T_DP + rd * 64 + c * 32, u);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc[c * 32 + e] = __uint_as_float(u[e]);
+          }
+          tmem_ld_wait();
+          if (rd == HD / 64 - 1) {
+            tc_fence_before();
+            bar_arrive(dq_free);
+          }
+          if (rd > 0) {  // the previous round's boxes must have been read
+            if (q == 0) bulk_wait_read_all();
+            named_bar_sync(2, 128);
+          }
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            uint8_t* box = sDS + bb * 16384 + q * 128;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int c = bb * 32 + u * 4;
+              *reinterpret_cast<float4*>(box + ((u ^ (q & 7)) * 16)) =
+                  make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+            }
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(2, 128);
+          if (q == 0) {
+            tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sDS), rd * 64, i0, bh);
+            tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sDS + 16384), rd * 64 + 32, i0, bh);
+            bulk_commit();
+          }
+        }
+        if (q == 0) bulk_wait_read_all();
+        if (q == 0) bar_arrive(stage_free);
       }
-      tmem_ld_wait();
-      tc_fence_before();
-      bar_arrive(dq_free);
-      if (i < p.N) {
-        float* dst = p.dq_accum + (head_off + i) * HD;
-#pragma unroll
-        for (int c = 0; c < HD; c += 4) red_add_v4(dst + c, acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-      }
+      if (q == 0) bulk_wait_all();
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

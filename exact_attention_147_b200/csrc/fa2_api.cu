@@ -138,6 +138,21 @@ fa2_status encode_bf16_4d(CUtensorMap* m, const void* ptr, const fa2_strides& s,
   return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
 }
 
+// 3-D map over the fp32 dQ accumulator [B*H, N, d] (dense): dims (d, N, B*H),
+// box (32, 128, 1), 128-byte swizzle; used for TMA bulk reductions.
+fa2_status encode_dqacc_3d(CUtensorMap* m, void* ptr, int B, int N, int H, int d) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  FA2_TRY(get_encoder(&enc));
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(B) * cuuint64_t(H)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(N) * cuuint64_t(d) * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
+}
+
 Strides to_s(const fa2_strides& s) { return Strides{s.b, s.n, s.h}; }
 
 void normalise_window(int causal, int* wl, int* wr) {
@@ -202,6 +217,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   FA2_TRY(encode_bf16_4d(&p.tm_dq, a.dq, sdq, a.B, a.N, a.H, HD, 128));
   FA2_TRY(encode_bf16_4d(&p.tm_dk, a.dk, sdk, a.B, a.N, a.H, HD, 128));
   FA2_TRY(encode_bf16_4d(&p.tm_dv, a.dv, sdv, a.B, a.N, a.H, HD, 128));
+  if (!deterministic) FA2_TRY(encode_dqacc_3d(&p.tm_dqacc, a.dq_accum, a.B, a.N, a.H, HD));
   p.lse = a.lse;
   p.dvec = a.dvec;
   p.dq_accum = a.dq_accum;
@@ -218,6 +234,17 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.wait_ns = g_wait_ns.load();
   const unsigned grid = unsigned(p.nblocks) * unsigned(a.H) * unsigned(a.B);
   constexpr int smem1 = BwdCfg<HD>::SMEM_BYTES;
+  // Kernel 1 re-balances registers between its warpgroups; the shares add up
+  // to 512 threads x REGS_AT_LAUNCH, so the compiled kernel must launch with
+  // at least that many registers per thread, or the increase would wait
+  // forever.  Refuse to launch otherwise.
+  {
+    cudaFuncAttributes fa;
+    auto k1c = deterministic ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false>
+                             : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true>;
+    if (cudaFuncGetAttributes(&fa, k1c) != cudaSuccess) return FA2_ERR_CUDA;
+    if (fa.numRegs < BwdCfg<HD>::REGS_AT_LAUNCH) return FA2_ERR_UNSUPPORTED;
+  }
   if (!deterministic) {
     const long long n4 = (long long)a.B * a.H * a.N * HD / 4;
     const unsigned zgrid = unsigned(std::min<long long>((n4 + 255) / 256, 148 * 16));

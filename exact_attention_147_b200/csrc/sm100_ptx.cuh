@@ -79,8 +79,9 @@ struct AbortFlag {
 // itself sleeps for a short, hardware-chosen time) and checks the clock
 // every 64 polls.  Returns false, after recording `site` in the device
 // status word, if `limit_ns` nanoseconds pass or another role has already
-// aborted.
-__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, AbortFlag ab,
+// aborted.  Inlined: a real call would fix one register budget for every
+// caller, which kernels that re-balance registers per warpgroup cannot use.
+__device__ __forceinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, AbortFlag ab,
                                            uint64_t limit_ns, int site) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -128,6 +129,17 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
       : "memory");
 }
 
+// Element-wise add of a shared-memory box into global memory through a
+// tensor map (the data type comes from the map).
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int c0, int c1,
+                                                  int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::
+          "l"(reinterpret_cast<uint64_t>(tmap)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -148,6 +160,21 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // Named barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier that also returns whether `pred` holds in every
+// participating thread (so a group can leave a loop together).
+__device__ __forceinline__ bool named_bar_all(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.eq.u32 p, %3, 0;\n\t"
+      "bar.red.or.pred q, %1, %2, p;\n\t"
+      "selp.u32 %0, 0, 1, q;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(count), "r"(pred ? 1u : 0u)
+      : "memory");
+  return r != 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -291,6 +318,21 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Register re-balancing between warpgroups.  All four warps of a warpgroup
+// execute the same instruction.  The CTA's pool is what it was launched
+// with (threads x registers at launch), so the per-warpgroup targets must
+// add up to no more than that.
+// ---------------------------------------------------------------------------
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------------------
