@@ -73,11 +73,16 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + Q_STAGES * TILE;
   static constexpr int OFF_DS = OFF_DO + DO_STAGES * TILE;
   static constexpr int OFF_SIDE = OFF_DS + DS_BYTES;
-  static constexpr int OFF_BARS = OFF_SIDE + Q_STAGES * SIDE_BYTES;
+  static constexpr int OFF_STG = OFF_SIDE + Q_STAGES * SIDE_BYTES;  // dQ staging ring
+  static constexpr int STG_BYTES = 2 * 16384;                         // 2 x (128 rows x 32 fp32)
+  static constexpr int OFF_BARS = OFF_STG + STG_BYTES;
   // kv_full, Q full/empty, dO full/empty, s_full, dp_full, p_ready, ds_ready,
-  // dq_full, dq_free, acc_full, stage_free, drain
-  static constexpr int NBARS = 1 + 2 * Q_STAGES + 2 * DO_STAGES + 9;
-  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16 + 1024;
+  // dq_full, dq_free, acc_full, drain
+  static constexpr int NBARS = 1 + 2 * Q_STAGES + 2 * DO_STAGES + 8;
+  // No alignment slack: the kernel checks that the dynamic shared memory
+  // starts on a 1024-byte boundary (it does: the reserved 1 KB precedes it).
+  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static constexpr int THREADS = 512;
   // registers per thread after the warpgroup re-balancing (see kernel 1)
   static constexpr int REGS_COMPUTE = 176, REGS_DRAIN = 96, REGS_MISC = 64;
@@ -102,6 +107,7 @@ namespace bwd_detail {
 constexpr float LOG2E = 1.44269504088896340736f;
 constexpr int SITE_BPROD = 0x500, SITE_BMMA = 0x600, SITE_BCOMP = 0x700, SITE_BRED = 0x800;
 constexpr int SITE_QPROD = 0x900, SITE_QMMA = 0xA00, SITE_QCOMP = 0xB00;
+constexpr int SITE_SMEM_ALIGN = 0xF00;
 
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
@@ -147,14 +153,18 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   constexpr int NCH = HD / 64;
   constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + HD;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // 128-byte-swizzled tiles need 1 KB alignment
+    if (threadIdx.x == 0) atomicCAS(&g_fa2_device_status, 0, SITE_SMEM_ALIGN);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sDO = smem + C::OFF_DO;
   uint8_t* sDS = smem + C::OFF_DS;
+  uint8_t* sStg = smem + C::OFF_STG;
   float* sSide = reinterpret_cast<float*>(smem + C::OFF_SIDE);  // [QS][2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
   const uint32_t b0 = smem_u32(bars);
@@ -166,7 +176,6 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   const uint32_t s_full = b0 + 8u * (1 + 2 * QS + 2 * DS);
   const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24;
   const uint32_t dq_full = s_full + 32, dq_free = s_full + 40, acc_full = s_full + 48;
-  const uint32_t stage_free = s_full + 56;
   const uint32_t drain_bar = b0 + 8u * (C::NBARS - 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
@@ -423,8 +432,6 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       bar_arrive(p_ready);
       // dS^T = P^T o (dP^T - D), 32 columns at a time
       ok = wait_bar(dp_full, it & 1, ab, p.wait_ns, SITE_BCOMP + 1);
-      // the dS^T tile doubles as the dQ staging buffer of the previous block
-      if (WITH_DQ && it > 0 && ok) ok = wait_bar(stage_free, (it - 1) & 1, ab, p.wait_ns, SITE_BCOMP + 3);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -496,49 +503,53 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         // leave together: the rounds below use a warpgroup-wide barrier
         if (!named_bar_all(2, 128, ok)) break;
         tc_fence_after();
-        // 64 columns per round: read them from TMEM, stage them as two
-        // 32-column (128-byte) swizzled boxes of 128 rows in the dS^T tile,
-        // and add each box into the accumulator with one bulk reduction.
-        // TMEM is released as soon as the last round's columns are read.
+        // dQ leaves TMEM 32 columns (one 128-byte swizzled box of 128 rows)
+        // at a time and is added into the accumulator with one TMA bulk
+        // reduction per box, staged through a two-slot ring.  Chunks 0..1
+        // go out right away; the remaining chunks are read into registers
+        // before TMEM is released, then staged as their slots free up.
+        auto stage = [&](const uint32_t (&u)[32], int chunk) {
+          if (q == 0) bulk_wait_read_1();   // the slot's previous box has been read
+          named_bar_sync(2, 128);
+          uint8_t* row = sStg + (chunk & 1) * 16384 + q * 128;
 #pragma unroll
-        for (int rd = 0; rd < HD / 64; ++rd) {
-          float acc[64];
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t u[32];
-            tmem_ld32(tmem + lane_base + T_DP + rd * 64 + c * 32, u);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) acc[c * 32 + e] = __uint_as_float(u[e]);
-          }
-          tmem_ld_wait();
-          if (rd == HD / 64 - 1) {
-            tc_fence_before();
-            bar_arrive(dq_free);
-          }
-          if (rd > 0) {  // the previous round's boxes must have been read
-            if (q == 0) bulk_wait_read_all();
-            named_bar_sync(2, 128);
-          }
-#pragma unroll
-          for (int bb = 0; bb < 2; ++bb) {
-            uint8_t* box = sDS + bb * 16384 + q * 128;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int c = bb * 32 + u * 4;
-              *reinterpret_cast<float4*>(box + ((u ^ (q & 7)) * 16)) =
-                  make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-            }
-          }
+          for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<uint4*>(row + ((e ^ (q & 7)) * 16)) =
+                make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
           fence_proxy_async_smem();
           named_bar_sync(2, 128);
           if (q == 0) {
-            tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sDS), rd * 64, i0, bh);
-            tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sDS + 16384), rd * 64 + 32, i0, bh);
+            tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sStg + (chunk & 1) * 16384), chunk * 32, i0, bh);
             bulk_commit();
           }
+        };
+        constexpr int NC = HD / 32;
+        {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_base + T_DP + 0, u);
+          tmem_ld_wait();
+          stage(u, 0);
         }
-        if (q == 0) bulk_wait_read_all();
-        if (q == 0) bar_arrive(stage_free);
+        {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_base + T_DP + 32, u);
+          tmem_ld_wait();
+          if (NC == 2) {
+            tc_fence_before();
+            bar_arrive(dq_free);
+          }
+          stage(u, 1);
+        }
+        if (NC == 4) {
+          uint32_t u2[32], u3[32];
+          tmem_ld32(tmem + lane_base + T_DP + 64, u2);
+          tmem_ld32(tmem + lane_base + T_DP + 96, u3);
+          tmem_ld_wait();
+          tc_fence_before();
+          bar_arrive(dq_free);
+          stage(u2, 2);
+          stage(u3, 3);
+        }
       }
       if (q == 0) bulk_wait_all();
     }
