@@ -85,7 +85,7 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static constexpr int THREADS = 512;
   // registers per thread after the warpgroup re-balancing (see kernel 1)
-  static constexpr int REGS_COMPUTE = 176, REGS_DRAIN = 96, REGS_MISC = 64;
+  static constexpr int REGS_COMPUTE = 144, REGS_DRAIN = 160, REGS_MISC = 64;
   static constexpr int REGS_AT_LAUNCH = (2 * 128 * REGS_COMPUTE + 128 * REGS_DRAIN + 128 * REGS_MISC) / 512;
   static_assert(REGS_AT_LAUNCH == 128, "register split must use exactly the launch budget");
 };
@@ -135,15 +135,15 @@ __device__ __forceinline__ void st_sw128_row32(uint8_t* tile, int row, int col0,
 // 16 warps: warpgroups 0 and 1 compute (thread = key row; warpgroup w owns
 // query columns [64w, 64w+64) of every S^T / dP^T tile), warpgroup 2 drains
 // dQ (thread = query row), warp 12 loads, warp 13 issues the MMAs.  Register
-// budget after the split: compute 176, drain 96, loader/MMA warpgroup 64
-// (2*128*176 + 128*96 + 128*64 = 65536 = 512 threads x 128 at launch; the
+// budget after the split: compute 144, drain 160, loader/MMA warpgroup 64
+// (2*128*144 + 128*160 + 128*64 = 65536 = 512 threads x 128 at launch; the
 // host checks the launch register count before every launch).
 //
-// dQ path: the drain warpgroup reads the dQ tile out of TMEM 64 columns at
-// a time, stages each round in the dS^T tile of shared memory (free once the
-// dQ MMA is done) and adds it into the fp32 accumulator with TMA bulk
-// reductions, which go through the TMA unit rather than the load/store
-// queues.  TMEM is released after the last round is read.
+// dQ path: the drain warpgroup reads the whole dQ tile out of TMEM into
+// registers, releases the TMEM columns (the next dP^T reuses them), then
+// stages it 32 columns at a time through a two-slot shared-memory ring and
+// adds it into the fp32 accumulator with TMA bulk reductions, which go
+// through the TMA unit rather than the load/store queues.
 // ---------------------------------------------------------------------------
 template <int HD, bool ALIBI, bool WITH_DQ>
 __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
@@ -309,38 +309,51 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           umma_ts(d_tmem, a_tmem + 64 * (kk / 4) + (kk % 4) * 8,
                   sdesc_sw128(bb + kk * 2048, 16384, 1024), id_pd, (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_bar(kv_full, 0, ab, p.wait_ns, SITE_BMMA + 0);
-      if (ok) ok = wait_bar(q_full(0), 0, ab, p.wait_ns, SITE_BMMA + 1);
-      tc_fence_after();
-      if (ok) {
-        kmajor(tmem + T_S, sK, sQ);
-        umma_commit(s_full);
-      }
-      for (int it = 0; it < nq && ok; ++it) {
-        const int sq = it % QS, sd = it % DS;
-        ok = wait_bar(do_full(sd), (it / DS) & 1, ab, p.wait_ns, SITE_BMMA + 2);
-        if (ok && WITH_DQ && it > 0) ok = wait_bar(dq_free, (it - 1) & 1, ab, p.wait_ns, SITE_BMMA + 3);
-        if (!ok) break;
+      // Issue order.  Prologue: S_0, dP_0, dV_0, S_1.  Then for block i:
+      //   dK_i, dQ_i       (need dS_i)
+      //   dP_{i+1}         (needs dQ_i drained out of the shared TMEM columns;
+      //                     runs while the compute warps form P_{i+1})
+      //   dV_{i+1}         (needs P_{i+1})
+      //   S_{i+2}          (S columns are free once dV_{i+1} has read P_{i+1})
+      // The compute warps work in the order P_0, dS_0, P_1, dS_1, ...
+      auto dp = [&](int k) {                      // dP_k^T = V dO_k^T
+        const int sd = k % DS;
+        if (!wait_bar(do_full(sd), (k / DS) & 1, ab, p.wait_ns, SITE_BMMA + 2)) return false;
+        if (WITH_DQ && k > 0 && !wait_bar(dq_free, (k - 1) & 1, ab, p.wait_ns, SITE_BMMA + 3))
+          return false;
         tc_fence_after();
-        kmajor(tmem + T_DP, sV, sDO + sd * C::TILE);                      // dP^T = V dO^T
+        kmajor(tmem + T_DP, sV, sDO + sd * C::TILE);
         umma_commit(dp_full);
-        ok = wait_bar(p_ready, it & 1, ab, p.wait_ns, SITE_BMMA + 4);
-        if (!ok) break;
+        return true;
+      };
+      auto dv = [&](int k, bool acc) {            // dV += P_k^T dO_k
+        const int sd = k % DS;
+        if (!wait_bar(p_ready, k & 1, ab, p.wait_ns, SITE_BMMA + 4)) return false;
         tc_fence_after();
-        from_tmem(tmem + T_DV, tmem + T_S, sDO + sd * C::TILE, it > 0);  // dV += P^T dO
+        from_tmem(tmem + T_DV, tmem + T_S, sDO + sd * C::TILE, acc);
         umma_commit(do_empty(sd));
-        if (it + 1 < nq) {
-          const int sn = (it + 1) % QS;
-          ok = wait_bar(q_full(sn), ((it + 1) / QS) & 1, ab, p.wait_ns, SITE_BMMA + 5);
-          if (!ok) break;
-          tc_fence_after();
-          kmajor(tmem + T_S, sK, sQ + sn * C::TILE);                     // next S^T
-          umma_commit(s_full);
-        }
+        return true;
+      };
+      auto s_next = [&](int k) {                  // S_k^T = K Q_k^T
+        const int sn = k % QS;
+        if (!wait_bar(q_full(sn), (k / QS) & 1, ab, p.wait_ns, SITE_BMMA + 5)) return false;
+        tc_fence_after();
+        kmajor(tmem + T_S, sK, sQ + sn * C::TILE);
+        umma_commit(s_full);
+        return true;
+      };
+      bool ok = wait_bar(kv_full, 0, ab, p.wait_ns, SITE_BMMA + 0);
+      ok = ok && s_next(0);
+      ok = ok && dp(0);
+      ok = ok && dv(0, false);
+      if (ok && nq > 1) ok = s_next(1);
+      for (int it = 0; it < nq && ok; ++it) {
+        const int sq = it % QS;
         ok = wait_bar(ds_ready, it & 1, ab, p.wait_ns, SITE_BMMA + 6);
         if (!ok) break;
         tc_fence_after();
-        from_tmem(tmem + T_DK, tmem + T_DP, sQ + sq * C::TILE, it > 0);  // dK += dS^T Q
+        from_tmem(tmem + T_DK, tmem + T_DP, sQ + sq * C::TILE, it > 0);   // dK += dS^T Q
+        umma_commit(q_empty(sq));
         if (WITH_DQ) {
           // dQ_i = dS K: A = dS (queries x keys) read MN-major from the dS^T
           // tile, B = K (keys x d) MN-major.
@@ -349,9 +362,10 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           for (int kk = 0; kk < 128 / 16; ++kk)
             umma_ss(tmem + T_DP, sdesc_sw128(a0 + kk * 2048, 16384, 1024),
                     sdesc_sw128(kb0 + kk * 2048, 16384, 1024), id_dq, kk > 0);
+          umma_commit(dq_full);
         }
-        umma_commit(q_empty(sq));
-        if (WITH_DQ) umma_commit(dq_full);
+        if (it + 1 < nq) ok = dp(it + 1) && dv(it + 1, true);
+        if (ok && it + 2 < nq) ok = s_next(it + 2);
       }
       umma_commit(acc_full);
       umma_commit(drain_bar);
@@ -382,35 +396,34 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       if (!ok) break;
       tc_fence_after();
       float pr[64];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_base + T_S + cq + c * 32, u);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pr[c * 32 + e] = __uint_as_float(u[e]);
-      }
-      tmem_ld_wait();
       const bool full = (i0 >= lo_q) && (i0 + 63 <= hi_q);
       const float fj = float(i0 - j);
 #pragma unroll
-      for (int c = 0; c < 64; c += 4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(side + c);
-        float x0, x1, x2, x3;
-        if (ALIBI) {
-          x0 = fmaf(slope2, fabsf(fj + float(c)), fmaf(pr[c], C2, -l4.x));
-          x1 = fmaf(slope2, fabsf(fj + float(c + 1)), fmaf(pr[c + 1], C2, -l4.y));
-          x2 = fmaf(slope2, fabsf(fj + float(c + 2)), fmaf(pr[c + 2], C2, -l4.z));
-          x3 = fmaf(slope2, fabsf(fj + float(c + 3)), fmaf(pr[c + 3], C2, -l4.w));
-        } else {
-          x0 = fmaf(pr[c], C2, -l4.x);
-          x1 = fmaf(pr[c + 1], C2, -l4.y);
-          x2 = fmaf(pr[c + 2], C2, -l4.z);
-          x3 = fmaf(pr[c + 3], C2, -l4.w);
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + T_S + cq + h2 * 32, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const int c = h2 * 32 + e;
+          const float4 l4 = *reinterpret_cast<const float4*>(side + c);
+          float x0, x1, x2, x3;
+          if (ALIBI) {
+            x0 = fmaf(slope2, fabsf(fj + float(c)), fmaf(__uint_as_float(u[e]), C2, -l4.x));
+            x1 = fmaf(slope2, fabsf(fj + float(c + 1)), fmaf(__uint_as_float(u[e + 1]), C2, -l4.y));
+            x2 = fmaf(slope2, fabsf(fj + float(c + 2)), fmaf(__uint_as_float(u[e + 2]), C2, -l4.z));
+            x3 = fmaf(slope2, fabsf(fj + float(c + 3)), fmaf(__uint_as_float(u[e + 3]), C2, -l4.w));
+          } else {
+            x0 = fmaf(__uint_as_float(u[e]), C2, -l4.x);
+            x1 = fmaf(__uint_as_float(u[e + 1]), C2, -l4.y);
+            x2 = fmaf(__uint_as_float(u[e + 2]), C2, -l4.z);
+            x3 = fmaf(__uint_as_float(u[e + 3]), C2, -l4.w);
+          }
+          pr[c] = ex2(x0);
+          pr[c + 1] = ex2(x1);
+          pr[c + 2] = ex2(x2);
+          pr[c + 3] = ex2(x3);
         }
-        pr[c] = ex2(x0);
-        pr[c + 1] = ex2(x1);
-        pr[c + 2] = ex2(x2);
-        pr[c + 3] = ex2(x3);
       }
       if (!full) {
 #pragma unroll
@@ -442,10 +455,13 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 16; e += 2) {
           const int cc = c * 32 + 2 * e;
-          w[e] = pack_bf16(pr[cc] * (__uint_as_float(u[2 * e]) - side[128 + cc]),
-                           pr[cc + 1] * (__uint_as_float(u[2 * e + 1]) - side[128 + cc + 1]));
+          const float4 d4 = *reinterpret_cast<const float4*>(side + 128 + cc);
+          w[e] = pack_bf16(pr[cc] * (__uint_as_float(u[2 * e]) - d4.x),
+                           pr[cc + 1] * (__uint_as_float(u[2 * e + 1]) - d4.y));
+          w[e + 1] = pack_bf16(pr[cc + 2] * (__uint_as_float(u[2 * e + 2]) - d4.z),
+                               pr[cc + 3] * (__uint_as_float(u[2 * e + 3]) - d4.w));
         }
         // written over columns this thread has already read
         tmem_st16(tmem + lane_base + T_DP + cq + c * 16, w);
@@ -491,7 +507,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       bulk_wait_all();
     }
   } else {
-    regs_dec<C::REGS_DRAIN>();
+    regs_inc<C::REGS_DRAIN>();
     if (WITH_DQ) {
       // ---------------------------------------------------------- dQ drain (query rows)
       const int q = (warp % 4) * 32 + lane;
@@ -524,32 +540,14 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           }
         };
         constexpr int NC = HD / 32;
-        {
-          uint32_t u[32];
-          tmem_ld32(tmem + lane_base + T_DP + 0, u);
-          tmem_ld_wait();
-          stage(u, 0);
-        }
-        {
-          uint32_t u[32];
-          tmem_ld32(tmem + lane_base + T_DP + 32, u);
-          tmem_ld_wait();
-          if (NC == 2) {
-            tc_fence_before();
-            bar_arrive(dq_free);
-          }
-          stage(u, 1);
-        }
-        if (NC == 4) {
-          uint32_t u2[32], u3[32];
-          tmem_ld32(tmem + lane_base + T_DP + 64, u2);
-          tmem_ld32(tmem + lane_base + T_DP + 96, u3);
-          tmem_ld_wait();
-          tc_fence_before();
-          bar_arrive(dq_free);
-          stage(u2, 2);
-          stage(u3, 3);
-        }
+        uint32_t u[NC][32];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32(tmem + lane_base + T_DP + c * 32, u[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        bar_arrive(dq_free);   // TMEM columns may now take the next dP^T
+#pragma unroll
+        for (int c = 0; c < NC; ++c) stage(u[c], c);
       }
       if (q == 0) bulk_wait_all();
     }
