@@ -46,7 +46,7 @@ namespace fa2 {
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;   // inputs, box {64,1,128,1}
   CUtensorMap tm_dq, tm_dk, tm_dv;       // outputs (bf16), same boxes
-  CUtensorMap tm_dqacc;                  // fp32 [B*H, N, d] accumulator, box {32,128,1}
+  CUtensorMap tm_dqacc;                  // fp32 [B*H, N, d] accumulator, box {32,32,1}
   const float* lse;                      // [B,H,N]
   const float* dvec;                     // [B,H,N]
   float* dq_accum;                       // [B,H,N,d] fp32 (kernel 1 with dQ)
@@ -516,26 +516,29 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       for (int it = 0; it < nq; ++it) {
         const int i0 = (qb_begin + it) * 128;
         bool ok = wait_bar(dq_full, it & 1, ab, p.wait_ns, SITE_BRED);
-        // leave together: the rounds below use a warpgroup-wide barrier
-        if (!named_bar_all(2, 128, ok)) break;
+        if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
         // dQ leaves TMEM 32 columns (one 128-byte swizzled box of 128 rows)
         // at a time and is added into the accumulator with one TMA bulk
         // reduction per box, staged through a two-slot ring.  Chunks 0..1
         // go out right away; the remaining chunks are read into registers
         // before TMEM is released, then staged as their slots free up.
+        // Each warp stages its own 32 rows (a 32 x 32-column box, 4 KB) and
+        // issues the bulk reduction for them: no cross-warp barrier.
+        const int wq = warp % 4;
         auto stage = [&](const uint32_t (&u)[32], int chunk) {
-          if (q == 0) bulk_wait_read_1();   // the slot's previous box has been read
-          named_bar_sync(2, 128);
+          if (lane == 0) bulk_wait_read_1();   // this warp's previous box in the slot was read
+          __syncwarp();
           uint8_t* row = sStg + (chunk & 1) * 16384 + q * 128;
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             *reinterpret_cast<uint4*>(row + ((e ^ (q & 7)) * 16)) =
                 make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
           fence_proxy_async_smem();
-          named_bar_sync(2, 128);
-          if (q == 0) {
-            tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sStg + (chunk & 1) * 16384), chunk * 32, i0, bh);
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sStg + (chunk & 1) * 16384 + wq * 4096), chunk * 32,
+                              i0 + wq * 32, bh);
             bulk_commit();
           }
         };
@@ -549,7 +552,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
 #pragma unroll
         for (int c = 0; c < NC; ++c) stage(u[c], c);
       }
-      if (q == 0) bulk_wait_all();
+      if (lane == 0) bulk_wait_all();
     }
   }
 

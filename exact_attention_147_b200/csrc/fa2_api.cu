@@ -139,13 +139,14 @@ fa2_status encode_bf16_4d(CUtensorMap* m, const void* ptr, const fa2_strides& s,
 }
 
 // 3-D map over the fp32 dQ accumulator [B*H, N, d] (dense): dims (d, N, B*H),
-// box (32, 128, 1), 128-byte swizzle; used for TMA bulk reductions.
+// box (32, 32, 1) -- one warp's 32 rows -- 128-byte swizzle; used for TMA
+// bulk reductions.
 fa2_status encode_dqacc_3d(CUtensorMap* m, void* ptr, int B, int N, int H, int d) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   FA2_TRY(get_encoder(&enc));
   cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(B) * cuuint64_t(H)};
   cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(N) * cuuint64_t(d) * 4};
-  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t box[3] = {32, 32, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
