@@ -388,8 +388,8 @@ def run_gpu(args):
                                     if k2 in ("value", "unit", "cores", "kind", "sample")}
         except Exception as ex:  # pragma: no cover
             line["cpu_baseline"] = {"error": str(ex)}
-    if args.sweep and world == 1:
-        line["sweep"] = run_sweep(F, W, args)
+    if world == 1 and not args.no_by_n:
+        line["by_n"] = run_sweep(F, W, args, full=args.sweep)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -398,12 +398,13 @@ def run_gpu(args):
     return 0
 
 
-def run_sweep(F, W, args):
+def run_sweep(F, W, args, full=False):
     """TFLOP/s of fwd and bwd (timed separately) over the sequence-length
-    sweep at 16384 tokens per batch, both head splits, causal and not."""
+    sweep at 16384 tokens per batch: hidden 2048 as H=16 x d=128 (and, with
+    --sweep, also H=32 x d=64), non-causal and causal."""
     import torch
     res = []
-    for d in (128, 64):
+    for d in ((128, 64) if full else (128,)):
         for n in W.SWEEP_N:
             for causal in (False, True):
                 w = W.sweep(n, d, causal)
@@ -431,8 +432,9 @@ def run_sweep(F, W, args):
                 tf = ev[0].elapsed_time(ev[1]) / reps
                 tb = ev[1].elapsed_time(ev[2]) / reps
                 res.append({"N": n, "d": d, "H": w.H, "B": w.B, "causal": causal,
-                            "fwd_ms": tf, "fwd_tflops": ff / (tf * 1e-3) / 1e12,
-                            "bwd_ms": tb, "bwd_tflops": 2.5 * ff / (tb * 1e-3) / 1e12})
+                            "fwd_ms": round(tf, 4), "fwd_tflops": round(ff / (tf * 1e-3) / 1e12, 1),
+                            "bwd_ms": round(tb, 4),
+                            "bwd_tflops": round(2.5 * ff / (tb * 1e-3) / 1e12, 1)})
                 del q, k, v, do, out, lse, D, dq, dk, dv, ws
                 torch.cuda.empty_cache()
     return res
@@ -444,7 +446,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libfa2", choices=["libfa2", "reference"])
-    ap.add_argument("--sweep", action="store_true", help="add the sequence-length sweep")
+    ap.add_argument("--sweep", action="store_true",
+                    help="extend the by-N table with the H=32 x d=64 split")
+    ap.add_argument("--no-by-n", action="store_true", help="skip the by-N table")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

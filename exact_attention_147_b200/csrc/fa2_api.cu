@@ -73,6 +73,7 @@ fa2_status check_options(float softmax_scale, float dropout_p, const float* alib
 struct DeviceInfo {
   int sm_major = -1;
   int sm_minor = -1;
+  int sm_count = 0;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -84,7 +85,8 @@ fa2_status current_device(int* dev, DeviceInfo* info) {
   DeviceInfo& di = g_dev[*dev];
   if (di.sm_major < 0) {
     if (cudaDeviceGetAttribute(&di.sm_major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&di.sm_minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess) {
+        cudaDeviceGetAttribute(&di.sm_minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess) {
       di.sm_major = -1;
       return FA2_ERR_CUDA;
     }
@@ -176,14 +178,17 @@ std::atomic<uint64_t> g_smem_fwd128{0}, g_smem_fwd128a{0}, g_smem_fwd64{0}, g_sm
 
 template <int HD, bool ALIBI>
 fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
-                            const fa2_strides& sv, const fa2_strides& so, int dev, int causal_order,
-                            cudaStream_t st, std::atomic<uint64_t>& mask) {
+                            const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
+                            int causal_order, cudaStream_t st, std::atomic<uint64_t>& mask) {
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
   FA2_TRY(encode_bf16_4d(&p.tm_q, a.q, sq, a.B, a.N, a.H, HD, 128));
   FA2_TRY(encode_bf16_4d(&p.tm_k, a.k, sk, a.B, a.N, a.H, HD, 128));
   FA2_TRY(encode_bf16_4d(&p.tm_v, a.v, sv, a.B, a.N, a.H, HD, 128));
-  FA2_TRY(encode_bf16_4d(&p.tm_o, a.o, so, a.B, a.N, a.H, HD, 128));
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.so_b = so.b;
+  p.so_n = so.n;
+  p.so_h = so.h;
   p.lse = a.lse;
   p.alibi = a.alibi;
   p.N = a.N;
@@ -192,13 +197,15 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.wl = a.wl;
   p.wr = a.wr;
   p.npairs = (a.N + 255) / 256;
+  p.num_units = p.npairs * a.H * a.B;
   p.heavy_first = causal_order;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.wait_ns = g_wait_ns.load();
   auto kern = fa2_fwd_sm100_kernel<HD, ALIBI>;
   constexpr int smem = FwdCfg<HD>::SMEM_BYTES;
   FA2_TRY(ensure_smem(kern, smem, dev, mask));
-  const unsigned grid = unsigned(p.npairs) * unsigned(a.H) * unsigned(a.B);
+  // persistent grid: one CTA per SM (shared memory and TMEM allow one)
+  const unsigned grid = unsigned(std::min(p.num_units, std::max(sm_count, 1)));
   kern<<<grid, FwdCfg<HD>::THREADS, smem, st>>>(p);
   return launched(1);
 }
@@ -346,11 +353,11 @@ fa2_status fa2_fwd(const void* q, const void* k, const void* v, void* o, float* 
   if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;  // sm_100a kernels only
   const int heavy_first = (a.wr >= 0 || a.wl >= 0) ? 1 : 0;
   if (d == 128) {
-    return alibi_slopes ? launch_fwd_sm100<128, true>(a, sq, sk, sv, so, dev, heavy_first, st, g_smem_fwd128a)
-                        : launch_fwd_sm100<128, false>(a, sq, sk, sv, so, dev, heavy_first, st, g_smem_fwd128);
+    return alibi_slopes ? launch_fwd_sm100<128, true>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st, g_smem_fwd128a)
+                        : launch_fwd_sm100<128, false>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st, g_smem_fwd128);
   }
-  return alibi_slopes ? launch_fwd_sm100<64, true>(a, sq, sk, sv, so, dev, heavy_first, st, g_smem_fwd64a)
-                      : launch_fwd_sm100<64, false>(a, sq, sk, sv, so, dev, heavy_first, st, g_smem_fwd64);
+  return alibi_slopes ? launch_fwd_sm100<64, true>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st, g_smem_fwd64a)
+                      : launch_fwd_sm100<64, false>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st, g_smem_fwd64);
 }
 
 fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D, int B, int N, int H, int d,

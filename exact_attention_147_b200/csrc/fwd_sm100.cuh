@@ -2,9 +2,12 @@
 //
 // Work split (FlashAttention-2 abstract, arXiv 2307.08691: parallelise over
 // thread blocks even within one head; FlashAttention-2 wiki article
-// "Technical architecture", improvement 2): each CTA owns a PAIR of 128-row
-// query tiles of one (batch, head), so the grid is (query pairs x heads x
-// batch) and a single long head already fills the GPU.
+// "Technical architecture", improvement 2): the unit of work is a PAIR of
+// 128-row query tiles of one (batch, head); the units (query pairs x heads x
+// batch) are ordered longest-first when masks make them uneven, and a
+// persistent grid of one CTA per SM walks them with a fixed stride, so a
+// single long head already fills the GPU and one unit's loads and first
+// products overlap the previous unit's epilogue.
 //
 // Inside a CTA (10 warps):
 //   warps 0-3   softmax for query tile 0 (thread = one query row)
@@ -14,6 +17,10 @@
 // The Q tiles stay resident in shared memory and K/V tiles stream through a
 // multi-slot TMA + mbarrier ring ("FlashAttention v2" article, §3.1-§3.2:
 // Q kept on chip, K/V prefetched while the current block is computed).
+//
+// The Q buffers are double-buffered across units; O leaves through registers
+// (normalised, cast to bf16 and stored by the row's own thread), so shared
+// memory holds only Q and the K/V ring.
 //
 // Tensor memory (512 columns x 128 lanes of fp32):
 //   [0,128)    S_0 (P_0 as bf16 pairs in its first 64 columns)
@@ -48,13 +55,16 @@
 namespace fa2 {
 
 struct FwdParams {
-  CUtensorMap tm_q, tm_k, tm_v, tm_o;  // [B,N,H,d] bf16, box {64,1,128,1}, 128B swizzle
+  CUtensorMap tm_q, tm_k, tm_v;        // [B,N,H,d] bf16, box {64,1,128,1}, 128B swizzle
+  __nv_bfloat16* o;                    // [B,N,H,d] output
+  long long so_b, so_n, so_h;          // its element strides
   float* lse;                          // [B,H,N]
   const float* alibi;                  // [H] or null
   int N, H, B;
   int wl, wr;                          // inclusive window, negative = unbounded
   int npairs;                          // ceil(N / 256)
-  int heavy_first;                     // order CTAs longest-first (causal)
+  int num_units;                       // npairs * H * B
+  int heavy_first;                     // order units longest-first (masks)
   float scale_log2;                    // softmax_scale * log2(e)
   unsigned long long wait_ns;          // bounded-wait limit
 };
@@ -63,13 +73,18 @@ template <int HD>
 struct FwdCfg {
   static constexpr int BM = 128;        // query rows per tile
   static constexpr int BN = 128;        // keys per KV block
-  static constexpr int NQT = 2;         // query tiles per CTA
-  static constexpr int SLOTS = HD == 128 ? 4 : 8;
+  static constexpr int NQT = 2;         // query tiles per unit
+  static constexpr int QBUFS = 2;       // Q double buffer (across units)
+  static constexpr int SLOTS = HD == 128 ? 3 : 8;
   static constexpr int QT_BYTES = BM * HD * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
-  // barriers: q_full, SLOTS x (full, empty), NQT x (s_full, p_ready, o_full), drain
-  static constexpr int NBARS = 1 + 2 * SLOTS + 3 * NQT + 1;
-  static constexpr int SMEM_BYTES = NQT * QT_BYTES + SLOTS * KV_BYTES + NBARS * 8 + 16 + 1024;
+  static constexpr int OFF_KV = QBUFS * NQT * QT_BYTES;
+  static constexpr int OFF_BARS = OFF_KV + SLOTS * KV_BYTES;
+  // q_full[2], q_empty[2], slot full/empty, s_full[2], p_ready[2], o_full[2],
+  // o_empty[2], drain
+  static constexpr int NBARS = 2 * QBUFS + 2 * SLOTS + 4 * NQT + 1;
+  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static constexpr int THREADS = 320;
 };
 
@@ -79,6 +94,39 @@ constexpr float LN2 = 0.69314718055994530942f;
 constexpr float LOG2E = 1.44269504088896340736f;
 // wait-site codes reported through the device status word
 constexpr int SITE_PROD = 0x100, SITE_MMA = 0x200, SITE_SOFT = 0x300, SITE_DRAIN = 0x400;
+constexpr int SITE_SMEM_ALIGN_F = 0xF01;
+
+// The k-th unit of CTA c in a persistent grid of G CTAs: round k covers
+// units [kG, kG + G) of the longest-first order, walked forwards in even
+// rounds and backwards in odd rounds, so each CTA's heavy and light units
+// pair up when the work per unit varies (causal and sliding-window masks).
+__device__ __forceinline__ int unit_index(int k) {
+  const int G = int(gridDim.x), c = int(blockIdx.x);
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
+}
+
+// Unit index -> (query pair, batch*H + head, first KV block, KV block count).
+struct Unit {
+  int pair, hb, row0, blk_begin, nblk;
+};
+__device__ __forceinline__ Unit unit_of(const FwdParams& p, int L) {
+  Unit u;
+  const int nhb = p.H * p.B;
+  if (p.heavy_first) {
+    u.pair = p.npairs - 1 - L / nhb;
+    u.hb = L % nhb;
+  } else {
+    u.pair = L % p.npairs;
+    u.hb = L / p.npairs;
+  }
+  u.row0 = u.pair * 256;
+  const int row_end = min(p.N, u.row0 + 256);
+  const int kv_lo = p.wl >= 0 ? max(0, u.row0 - p.wl) : 0;
+  const int kv_hi = p.wr >= 0 ? min(p.N - 1, row_end - 1 + p.wr) : p.N - 1;
+  u.blk_begin = kv_lo / 128;
+  u.nblk = kv_hi / 128 - u.blk_begin + 1;
+  return u;
+}
 }  // namespace fwd_detail
 
 // Bounded wait that ignores the CTA abort flag (used to drain in-flight
@@ -100,58 +148,38 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
   constexpr int NCH = HD / 64;  // 64-column (128-byte) boxes per tile row
   using namespace fwd_detail;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = smem + NQT * C::QT_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + SLOTS * C::KV_BYTES);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // 128-byte-swizzled tiles need 1 KB alignment
+    if (threadIdx.x == 0) atomicCAS(&g_fa2_device_status, 0, SITE_SMEM_ALIGN_F);
+    return;
+  }
+  uint8_t* sQ = smem_raw;                   // [QBUFS][NQT] tiles
+  uint8_t* sKV = smem_raw + C::OFF_KV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + C::OFF_BARS);
   const uint32_t bar0 = smem_u32(bars);
-  // barrier addresses
-  const uint32_t q_full = bar0;
-  auto slot_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto slot_empty = [&](int s) { return bar0 + 8u * (1 + SLOTS + s); };
-  auto s_full = [&](int t) { return bar0 + 8u * (1 + 2 * SLOTS + t); };
-  auto p_ready = [&](int t) { return bar0 + 8u * (3 + 2 * SLOTS + t); };
-  auto o_full = [&](int t) { return bar0 + 8u * (5 + 2 * SLOTS + t); };
-  const uint32_t drain_bar = bar0 + 8u * (7 + 2 * SLOTS);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * SLOTS);
+  auto q_full = [&](int qb) { return bar0 + 8u * qb; };
+  auto q_empty = [&](int qb) { return bar0 + 8u * (2 + qb); };
+  auto slot_full = [&](int s) { return bar0 + 8u * (4 + s); };
+  auto slot_empty = [&](int s) { return bar0 + 8u * (4 + SLOTS + s); };
+  auto s_full = [&](int t) { return bar0 + 8u * (4 + 2 * SLOTS + t); };
+  auto p_ready = [&](int t) { return bar0 + 8u * (6 + 2 * SLOTS + t); };
+  auto o_full = [&](int t) { return bar0 + 8u * (8 + 2 * SLOTS + t); };
+  auto o_empty = [&](int t) { return bar0 + 8u * (10 + 2 * SLOTS + t); };
+  const uint32_t drain_bar = bar0 + 8u * (12 + 2 * SLOTS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   AbortFlag ab{abort_flag};
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // Which (pair, head, batch) this CTA owns.
-  const int nhb = p.H * p.B;
-  int pair, hb;
-  if (p.heavy_first) {
-    pair = p.npairs - 1 - int(blockIdx.x / nhb);
-    hb = int(blockIdx.x % nhb);
-  } else {
-    pair = int(blockIdx.x % p.npairs);
-    hb = int(blockIdx.x / p.npairs);
-  }
-  const int h = hb % p.H, b = hb / p.H;
-  const int row0 = pair * (BM * NQT);
-  const int row_end = min(p.N, row0 + BM * NQT);
-  const int kv_lo = p.wl >= 0 ? max(0, row0 - p.wl) : 0;
-  const int kv_hi = p.wr >= 0 ? min(p.N - 1, row_end - 1 + p.wr) : p.N - 1;
-  const int blk_begin = kv_lo / BN;
-  const int nblk = kv_hi / BN - blk_begin + 1;
-
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    bar_init(q_full, 1);
-    for (int s = 0; s < SLOTS; ++s) {
-      bar_init(slot_full(s), 1);
-      bar_init(slot_empty(s), 1);
+    for (int i = 0; i < C::NBARS; ++i) {
+      const uint32_t bar = bar0 + 8u * i;
+      bar_init(bar, (bar == p_ready(0) || bar == p_ready(1) || bar == o_empty(0) || bar == o_empty(1))
+                        ? 128
+                        : 1);
     }
-    for (int t = 0; t < NQT; ++t) {
-      bar_init(s_full(t), 1);
-      bar_init(p_ready(t), 128);
-      bar_init(o_full(t), 1);
-    }
-    bar_init(drain_bar, 1);
     fence_barrier_init();
   }
   if (warp == 9) {
@@ -162,7 +190,6 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
-    tma_prefetch_desc(&p.tm_o);
   }
   tc_fence_before();
   __syncthreads();
@@ -172,40 +199,46 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      bar_arrive_expect_tx(q_full, NQT * C::QT_BYTES);
-      for (int t = 0; t < NQT; ++t)
-        for (int c = 0; c < NCH; ++c)
-          tma_load_4d(smem_u32(sQ + t * C::QT_BYTES + c * BM * 128), &p.tm_q, q_full, c * 64, h,
-                      row0 + t * BM, b);
-      int n = 0;
+      int n = 0, k = 0, q_issued = 0;
       bool ok = true;
-      for (int it = 0; it < nblk && ok; ++it) {
-        const int kv0 = (blk_begin + it) * BN;
-        for (int which = 0; which < 2; ++which, ++n) {
-          const int s = n % SLOTS;
-          if (!wait_bar(slot_empty(s), ((n / SLOTS) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + which)) {
-            ok = false;
-            break;
-          }
-          bar_arrive_expect_tx(slot_full(s), C::KV_BYTES);
-          const CUtensorMap* tm = which == 0 ? &p.tm_k : &p.tm_v;
+      for (int L = unit_index(0); L < p.num_units && ok; L = unit_index(++k)) {
+        const Unit u = unit_of(p, L);
+        const int h = u.hb % p.H, b = u.hb / p.H;
+        const int qb = k & 1;
+        if (!wait_bar(q_empty(qb), ((k >> 1) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + 2)) break;
+        bar_arrive_expect_tx(q_full(qb), NQT * C::QT_BYTES);
+        for (int t = 0; t < NQT; ++t)
           for (int c = 0; c < NCH; ++c)
-            tma_load_4d(smem_u32(sKV + s * C::KV_BYTES + c * BN * 128), tm, slot_full(s), c * 64, h,
-                        kv0, b);
+            tma_load_4d(smem_u32(sQ + (qb * NQT + t) * C::QT_BYTES + c * BM * 128), &p.tm_q, q_full(qb),
+                        c * 64, h, u.row0 + t * BM, b);
+        q_issued = k + 1;
+        for (int it = 0; it < u.nblk && ok; ++it) {
+          const int kv0 = (u.blk_begin + it) * BN;
+          for (int which = 0; which < 2; ++which, ++n) {
+            const int s = n % SLOTS;
+            if (!wait_bar(slot_empty(s), ((n / SLOTS) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + which)) {
+              ok = false;
+              break;
+            }
+            bar_arrive_expect_tx(slot_full(s), C::KV_BYTES);
+            const CUtensorMap* tm = which == 0 ? &p.tm_k : &p.tm_v;
+            for (int c = 0; c < NCH; ++c)
+              tma_load_4d(smem_u32(sKV + s * C::KV_BYTES + c * BN * 128), tm, slot_full(s), c * 64, h, kv0, b);
+          }
         }
       }
       // Before the CTA may exit, every copy issued must have landed.
-      drain_wait(q_full, 0, p.wait_ns);
-      for (int k = (n > SLOTS ? n - SLOTS : 0); k < n; ++k)
-        drain_wait(slot_full(k % SLOTS), (k / SLOTS) & 1, p.wait_ns);
+      for (int j = max(0, q_issued - 2); j < q_issued; ++j) drain_wait(q_full(j & 1), (j >> 1) & 1, p.wait_ns);
+      for (int j = (n > SLOTS ? n - SLOTS : 0); j < n; ++j)
+        drain_wait(slot_full(j % SLOTS), (j / SLOTS) & 1, p.wait_ns);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(BM, BN, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(BM, HD, 0, 1);
-      auto qk = [&](int t, int s) {
-        const uint32_t a0 = smem_u32(sQ + t * C::QT_BYTES), b0 = smem_u32(sKV + s * C::KV_BYTES);
+      auto qk = [&](int t, int qb, int s) {
+        const uint32_t a0 = smem_u32(sQ + (qb * NQT + t) * C::QT_BYTES), b0 = smem_u32(sKV + s * C::KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t ao = (kk / 4) * (BM * 128) + (kk % 4) * 32;
@@ -221,56 +254,67 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
           umma_ts(tmem + 256 + t * HD, tmem + t * 128 + kk * 8,
                   sdesc_sw128(v0 + kk * 2048, BN * 128, 1024), id_pv, (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_bar(q_full, 0, ab, p.wait_ns, SITE_MMA + 0);
-      tc_fence_after();
-      int n = 0;
-      if (ok) {
-        const int sk = n % SLOTS;
-        ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
-        tc_fence_after();
-        if (ok) {
+      int n = 0, k = 0, g = 0;  // KV slot counter, unit counter, block counter
+      bool ok = true;
+      for (int L = unit_index(0); L < p.num_units && ok; L = unit_index(++k)) {
+        const Unit u = unit_of(p, L);
+        const int qb = k & 1;
+        ok = wait_bar(q_full(qb), (k >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
+        if (!ok) break;
+        {
+          const int sk = n % SLOTS;
+          ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
+          if (!ok) break;
+          tc_fence_after();
           for (int t = 0; t < NQT; ++t) {
-            qk(t, sk);
+            qk(t, qb, sk);
             umma_commit(s_full(t));
           }
           umma_commit(slot_empty(sk));
+          if (u.nblk == 1) umma_commit(q_empty(qb));
           ++n;
         }
-      }
-      for (int it = 1; it < nblk && ok; ++it) {
-        const int sv = n % SLOTS, sk = (n + 1) % SLOTS;
-        ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
-        tc_fence_after();
-        for (int t = 0; t < NQT && ok; ++t) {
-          ok = wait_bar(p_ready(t), (it - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
-          tc_fence_after();
-          if (!ok) break;
-          pv(t, sv, it > 1);
-          if (t == 0) {
-            ok = wait_bar(slot_full(sk), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 4);
-            tc_fence_after();
+        for (int it = 1; it < u.nblk && ok; ++it) {
+          const int sv = n % SLOTS, sk = (n + 1) % SLOTS;
+          ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
+          for (int t = 0; t < NQT && ok; ++t) {
+            ok = wait_bar(p_ready(t), (g + it - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
+            // the first PV of a unit overwrites O_t: the previous unit's
+            // epilogue must have read it
+            if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
             if (!ok) break;
+            tc_fence_after();
+            pv(t, sv, it > 1);
+            if (t == 0) {
+              ok = wait_bar(slot_full(sk), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 4);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            qk(t, qb, sk);
+            umma_commit(s_full(t));
           }
-          qk(t, sk);
-          umma_commit(s_full(t));
+          if (!ok) break;
+          if (it == u.nblk - 1) umma_commit(q_empty(qb));  // the unit's last S products
+          umma_commit(slot_empty(sv));
+          umma_commit(slot_empty(sk));
+          n += 2;
         }
         if (!ok) break;
-        umma_commit(slot_empty(sv));
-        umma_commit(slot_empty(sk));
-        n += 2;
-      }
-      if (ok) {
-        const int sv = n % SLOTS;
-        ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 5);
-        tc_fence_after();
-        for (int t = 0; t < NQT && ok; ++t) {
-          ok = wait_bar(p_ready(t), (nblk - 1) & 1, ab, p.wait_ns, SITE_MMA + 6);
-          tc_fence_after();
-          if (!ok) break;
-          pv(t, sv, nblk > 1);
-          umma_commit(o_full(t));
+        {
+          const int sv = n % SLOTS;
+          ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 5);
+          for (int t = 0; t < NQT && ok; ++t) {
+            ok = wait_bar(p_ready(t), (g + u.nblk - 1) & 1, ab, p.wait_ns, SITE_MMA + 6);
+            if (ok && u.nblk == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+            if (!ok) break;
+            tc_fence_after();
+            pv(t, sv, u.nblk > 1);
+            umma_commit(o_full(t));
+          }
+          if (ok) umma_commit(slot_empty(sv));
+          ++n;
         }
-        if (ok) umma_commit(slot_empty(sv));
+        g += u.nblk;
       }
       // Drain: wait until every MMA issued above has completed.
       umma_commit(drain_bar);
@@ -280,145 +324,142 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
     // ------------------------------------------------------------ softmax
     const int t = warp / 4;
     const int r = (warp % 4) * 32 + lane;
-    const int i = row0 + t * BM + r;  // query row (>= N for padding rows)
     const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
     const uint32_t s_addr = tmem + lane_base + t * 128;
     const uint32_t o_addr = tmem + lane_base + 256 + t * HD;
-    const int lo = p.wl >= 0 ? max(0, i - p.wl) : 0;
-    const int hi = p.wr >= 0 ? min(p.N - 1, i + p.wr) : p.N - 1;
     const float C2 = p.scale_log2;
-    float slope2 = 0.f;
-    if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
-    float m_run = -CUDART_INF_F, l_run = 0.f;
+    int g = 0, k = 0;
     bool ok = true;
-    for (int it = 0; it < nblk; ++it) {
-      const int kv0 = (blk_begin + it) * BN;
-      ok = wait_bar(s_full(t), it & 1, ab, p.wait_ns, SITE_SOFT + 0);
+    for (int L = unit_index(0); L < p.num_units && ok; L = unit_index(++k)) {
+      const Unit u = unit_of(p, L);
+      const int h = u.hb % p.H, b = u.hb / p.H;
+      const int i = u.row0 + t * BM + r;  // query row (>= N for padding rows)
+      const int lo = p.wl >= 0 ? max(0, i - p.wl) : 0;
+      const int hi = p.wr >= 0 ? min(p.N - 1, i + p.wr) : p.N - 1;
+      float slope2 = 0.f;
+      if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
+      float m_run = -CUDART_INF_F, l_run = 0.f;
+      for (int it = 0; it < u.nblk; ++it) {
+        const int kv0 = (u.blk_begin + it) * BN;
+        ok = wait_bar(s_full(t), (g + it) & 1, ab, p.wait_ns, SITE_SOFT + 0);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        float s[BN];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t w32[32];
+          tmem_ld32(s_addr + c * 32, w32);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(w32[e]);
+        }
+        tmem_ld_wait();
+        if (ALIBI) {
+          const float fi = float(i - kv0);
+#pragma unroll
+          for (int c = 0; c < BN; ++c) s[c] = fmaf(slope2, fabsf(fi - float(c)), s[c] * C2);
+        }
+        if (!(kv0 >= lo && kv0 + BN - 1 <= hi)) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c) {
+            const int j = kv0 + c;
+            if (j < lo || j > hi) s[c] = -CUDART_INF_F;
+          }
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < BN; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        if (!ALIBI) mx *= C2;  // now in base-2 units
+        const bool resc = mx > m_run + TAU;
+        float alpha = 1.f;
+        if (resc) {
+          alpha = ex2(m_run - mx);  // 0 when m_run is -inf
+          m_run = mx;
+        }
+        const float m_use = m_run == -CUDART_INF_F ? 0.f : m_run;
+        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < BN; c += 4) {
+          if (ALIBI) {
+            s[c] = ex2(s[c] - m_use);
+            s[c + 1] = ex2(s[c + 1] - m_use);
+            s[c + 2] = ex2(s[c + 2] - m_use);
+            s[c + 3] = ex2(s[c + 3] - m_use);
+          } else {
+            s[c] = ex2(fmaf(s[c], C2, -m_use));
+            s[c + 1] = ex2(fmaf(s[c + 1], C2, -m_use));
+            s[c + 2] = ex2(fmaf(s[c + 2], C2, -m_use));
+            s[c + 3] = ex2(fmaf(s[c + 3], C2, -m_use));
+          }
+          l0 += s[c];
+          l1 += s[c + 1];
+          l2 += s[c + 2];
+          l3 += s[c + 3];
+        }
+        l_run = fmaf(l_run, alpha, (l0 + l1) + (l2 + l3));
+        // P (bf16 pairs) over the first BN/2 columns of S.
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t w16[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w16[e] = pack_bf16(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]);
+          tmem_st16(s_addr + c * 16, w16);
+        }
+        // Rescale the running output (the PV product of the previous block has
+        // completed: S_t of this block was committed after it).
+        if (it > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll
+          for (int c = 0; c < HD / 32; ++c) {
+            uint32_t w32[32];
+            tmem_ld32(o_addr + c * 32, w32);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) w32[e] = __float_as_uint(__uint_as_float(w32[e]) * alpha);
+            tmem_st32(o_addr + c * 32, w32);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        bar_arrive(p_ready(t));
+      }
+      if (!ok) break;
+      // -------------------------------------------------------- epilogue
+      ok = wait_bar(o_full(t), k & 1, ab, p.wait_ns, SITE_SOFT + 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      float s[BN];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(s_addr + c * 32, u);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(u[e]);
-      }
-      tmem_ld_wait();
-      if (ALIBI) {
-        const float fi = float(i - kv0);
-#pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = fmaf(slope2, fabsf(fi - float(c)), s[c] * C2);
-      }
-      if (!(kv0 >= lo && kv0 + BN - 1 <= hi)) {
-#pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const int j = kv0 + c;
-          if (j < lo || j > hi) s[c] = -CUDART_INF_F;
-        }
-      }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-      for (int c = 4; c < BN; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
-      }
-      float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-      if (!ALIBI) mx *= C2;  // now in base-2 units
-      const bool resc = mx > m_run + TAU;
-      float alpha = 1.f;
-      if (resc) {
-        alpha = ex2(m_run - mx);  // 0 when m_run is -inf
-        m_run = mx;
-      }
-      const float m_use = m_run == -CUDART_INF_F ? 0.f : m_run;
-      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-#pragma unroll
-      for (int c = 0; c < BN; c += 4) {
-        if (ALIBI) {
-          s[c] = ex2(s[c] - m_use);
-          s[c + 1] = ex2(s[c + 1] - m_use);
-          s[c + 2] = ex2(s[c + 2] - m_use);
-          s[c + 3] = ex2(s[c + 3] - m_use);
-        } else {
-          s[c] = ex2(fmaf(s[c], C2, -m_use));
-          s[c + 1] = ex2(fmaf(s[c + 1], C2, -m_use));
-          s[c + 2] = ex2(fmaf(s[c + 2], C2, -m_use));
-          s[c + 3] = ex2(fmaf(s[c + 3], C2, -m_use));
-        }
-        l0 += s[c];
-        l1 += s[c + 1];
-        l2 += s[c + 2];
-        l3 += s[c + 3];
-      }
-      l_run = fmaf(l_run, alpha, (l0 + l1) + (l2 + l3));
-      // P (bf16 pairs) over the first BN/2 columns of S.
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t u[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]);
-        tmem_st16(s_addr + c * 16, u);
-      }
-      // Rescale the running output (the PV product of the previous block has
-      // completed: S_t of this block was committed after it).
-      if (it > 0 && __any_sync(0xffffffffu, resc)) {
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32(o_addr + c * 32, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-          tmem_st32(o_addr + c * 32, u);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      bar_arrive(p_ready(t));
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok) ok = wait_bar(o_full(t), 0, ab, p.wait_ns, SITE_SOFT + 1);
-    ok = __all_sync(0xffffffffu, ok);
-    tc_fence_after();
-    uint8_t* stage = sQ + t * C::QT_BYTES;
-    if (ok) {
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      __nv_bfloat16* orow = p.o + b * p.so_b + (long long)i * p.so_n + h * p.so_h;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t w32[32];
+        tmem_ld32(o_addr + c * 32, w32);
+        tmem_ld_wait();
+        if (c == HD / 32 - 1) {  // O_t has been read: the next unit may overwrite it
+          tc_fence_before();
+          bar_arrive(o_empty(t));
+        }
+        uint32_t w16[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w16[e] = pack_bf16(__uint_as_float(w32[2 * e]) * inv_l, __uint_as_float(w32[2 * e + 1]) * inv_l);
+        if (i < p.N) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) =
+                make_uint4(w16[4 * q4], w16[4 * q4 + 1], w16[4 * q4 + 2], w16[4 * q4 + 3]);
+        }
+      }
       if (i < p.N)
         p.lse[(size_t(b) * p.H + h) * p.N + i] =
             l_run > 0.f ? (m_run + log2f(l_run)) * LN2 : -CUDART_INF_F;
-      // Stage O (bf16) in this tile's Q buffer, in the 128B-swizzled layout
-      // the O tensor map expects, then store it with TMA.
-#pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(o_addr + c * 32, u);
-        tmem_ld_wait();
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16(__uint_as_float(u[2 * e]) * inv_l, __uint_as_float(u[2 * e + 1]) * inv_l);
-        const int box = (c * 32) / 64;
-        const int u0 = ((c * 32) % 64) / 8;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint8_t* dst = stage + box * (BM * 128) + r * 128 + (((u0 + q4) ^ (r & 7)) * 16);
-          *reinterpret_cast<uint4*>(dst) =
-              make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-        }
-      }
-    }
-    // All 128 threads of the tile reach this barrier, on every path.
-    fence_proxy_async_smem();
-    named_bar_sync(1 + t, 128);
-    if (ok && r == 0 && row0 + t * BM < p.N) {
-      for (int c = 0; c < NCH; ++c)
-        tma_store_4d(&p.tm_o, smem_u32(stage + c * BM * 128), c * 64, h, row0 + t * BM, b);
-      bulk_commit();
-      bulk_wait_read_all();
+      g += u.nblk;
     }
   }
 
