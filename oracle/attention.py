@@ -41,6 +41,15 @@ Readings taken where the pages are silent (each repeated where it applies):
 * a row with no visible key (unreachable with the shipped masks, since the
   diagonal is always visible) has O = 0, LSE = -inf and zero gradients.
 
+Dropout (the call's ``dropout_p``; the pages give no formula, so the plain
+reading of attention dropout is taken): after the softmax, each probability
+is kept or zeroed by a given boolean mask and kept ones are multiplied by a
+given scale (1 / keep probability); O = (P o keep * scale) V, while LSE stays
+the log-sum-exp of the un-dropped scores.  The mask is an INPUT here (it is
+drawn by oracle/philox.py), so these functions hold no random-number code.
+In the backward pass the same mask multiplies dO V^T, and D = rowsum(dO o O)
+with the dropped O is still sum_j P_ij dP_ij.
+
 Layouts: q, k, v, o, do, dq, dk, dv are [B, N, H, d]; lse and D are
 [B, H, N].  All arithmetic is float64; callers pass the exact values the GPU
 receives (e.g. bf16 inputs widened to float64).
@@ -118,10 +127,13 @@ def _softmax_rows(s: np.ndarray):
 def head_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
                  causal: bool = False, window_left: int = -1,
                  window_right: int = -1, slope: float | None = None,
-                 rows: np.ndarray | None = None):
+                 rows: np.ndarray | None = None, keep=None,
+                 keep_scale: float = 1.0):
     """One head: q [Nq_rows, d] (the rows listed in ``rows``), k, v [N, d].
 
-    Returns (O [rows, d], LSE [rows]) with LSE = M + ln(l).
+    ``keep`` (optional): boolean [len(rows), N] dropout mask, applied to P
+    with ``keep_scale``.  Returns (O [rows, d], LSE [rows]) with
+    LSE = M + ln(l) of the un-dropped scores.
     """
     n = k.shape[0]
     if rows is None:
@@ -135,6 +147,8 @@ def head_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
         s = head_scores(q[r0:r0 + chunk], k, rr, scale, causal, window_left,
                         window_right, slope)
         p, m, l = _softmax_rows(s)
+        if keep is not None:
+            p = p * (keep[r0:r0 + chunk] * keep_scale)
         o[r0:r0 + chunk] = p @ v
         live = np.isfinite(m)
         lse[r0:r0 + chunk] = np.where(live, m + np.log(np.where(live, l, 1.0)),
@@ -145,12 +159,13 @@ def head_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
 def head_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
                   do: np.ndarray, scale: float, causal: bool = False,
                   window_left: int = -1, window_right: int = -1,
-                  slope: float | None = None):
+                  slope: float | None = None, keep=None,
+                  keep_scale: float = 1.0):
     """Textbook gradients for one head (q, k, v, do are [N, d]).
 
     The probabilities are recomputed from the inputs, as in the explainer's
-    "Backward pass" section.  Returns (dq, dk, dv, D) with D_i = sum_c
-    dO_ic O_ic.
+    "Backward pass" section.  ``keep``: optional [N, N] dropout mask (see the
+    module docstring).  Returns (dq, dk, dv, D) with D_i = sum_c dO_ic O_ic.
     """
     n, d = q.shape
     dq = np.zeros_like(q)
@@ -163,10 +178,12 @@ def head_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
         s = head_scores(q[rr], k, rr, scale, causal, window_left,
                         window_right, slope)
         p, _, _ = _softmax_rows(s)
-        o = p @ v
+        mk = 1.0 if keep is None else keep[rr] * keep_scale
+        pd = p * mk                            # dropped probabilities
+        o = pd @ v
         do_r = do[rr]
-        dv += p.T @ do_r                       # dV = P^T dO
-        dp = do_r @ v.T                        # dP = dO V^T
+        dv += pd.T @ do_r                      # dV = (P o keep)^T dO
+        dp = (do_r @ v.T) * mk                 # dP = (dO V^T) o keep
         d_r = np.sum(do_r * o, axis=1)         # D = rowsum(dO o O)
         ds = p * (dp - d_r[:, None])           # dS = P o (dP - D)
         dq[rr] = scale * (ds @ k)              # dQ = scale dS K
