@@ -3,6 +3,8 @@
 
 #include <cstdint>
 
+#include "philox.cuh"
+
 namespace fa2 {
 
 struct Strides {
@@ -29,6 +31,8 @@ struct AttnArgs {
   int B, N, H, d;
   float scale;        // softmax scale
   int wl, wr;         // window bounds, negative = unbounded
+  int dropout;        // nonzero: apply the dropout mask described in philox.cuh
+  DropoutParams drop;
 };
 
 // Keys visible to query i lie in [visible_lo, visible_hi] ("FlashAttention

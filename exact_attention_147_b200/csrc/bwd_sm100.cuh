@@ -39,6 +39,7 @@
 
 #include "attn_common.cuh"
 #include "fwd_sm100.cuh"
+#include "philox.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa2 {
@@ -58,6 +59,7 @@ struct BwdParams {
   float scale;                           // softmax scale c
   float scale_log2;                      // c * log2(e)
   unsigned long long wait_ns;
+  DropoutParams drop;                    // used by the DROPOUT instantiations
 };
 
 template <int HD>
@@ -145,7 +147,7 @@ __device__ __forceinline__ void st_sw128_row32(uint8_t* tile, int row, int col0,
 // adds it into the fp32 accumulator with TMA bulk reductions, which go
 // through the TMA unit rather than the load/store queues.
 // ---------------------------------------------------------------------------
-template <int HD, bool ALIBI, bool WITH_DQ>
+template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT>
 __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<HD>;
   using namespace bwd_detail;
@@ -432,12 +434,43 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           if (i < lo_q || i > hi_q) pr[c] = 0.f;
         }
       }
-      // P^T (bf16) into columns [cq, cq+32) of the S^T region (already read)
+      // Dropout: one generator call gives the bytes of this key for four
+      // consecutive queries (output word = query mod 4, byte = key mod 4).
+      uint32_t keep_lo = 0xFFFFFFFFu, keep_hi = 0xFFFFFFFFu;
+      if (DROPOUT) {
+        keep_lo = keep_hi = 0u;
+        const int jb = 8 * (j & 3);
+#pragma unroll
+        for (int a = 0; a < 16; ++a) {
+          const Philox4 o = philox4x32_10(uint32_t(j >> 2), uint32_t((i0 >> 2) + a), uint32_t(h),
+                                          uint32_t(b), p.drop.seed_lo, p.drop.seed_hi);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t kept = ((o.w[e] >> jb) & 0xFFu) >= p.drop.threshold ? 1u : 0u;
+            const int c = 4 * a + e;
+            if (c < 32) keep_lo |= kept << c;
+            else keep_hi |= kept << (c - 32);
+          }
+        }
+      }
+      auto kept = [&](int c) {
+        return ((c < 32 ? keep_lo >> c : keep_hi >> (c - 32)) & 1u) != 0u;
+      };
+      // P^T (bf16, dropped and rescaled when dropout is on) into columns
+      // [cq, cq+32) of the S^T region (already read)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) w[e] = pack_bf16(pr[c * 32 + 2 * e], pr[c * 32 + 2 * e + 1]);
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = c * 32 + 2 * e;
+          float a0 = pr[c0], a1 = pr[c0 + 1];
+          if (DROPOUT) {
+            a0 = kept(c0) ? a0 * p.drop.keep_scale : 0.f;
+            a1 = kept(c0 + 1) ? a1 * p.drop.keep_scale : 0.f;
+          }
+          w[e] = pack_bf16(a0, a1);
+        }
         tmem_st16(tmem + lane_base + T_S + cq + c * 16, w);
       }
       tmem_st_wait();
@@ -458,10 +491,16 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         for (int e = 0; e < 16; e += 2) {
           const int cc = c * 32 + 2 * e;
           const float4 d4 = *reinterpret_cast<const float4*>(side + 128 + cc);
-          w[e] = pack_bf16(pr[cc] * (__uint_as_float(u[2 * e]) - d4.x),
-                           pr[cc + 1] * (__uint_as_float(u[2 * e + 1]) - d4.y));
-          w[e + 1] = pack_bf16(pr[cc + 2] * (__uint_as_float(u[2 * e + 2]) - d4.z),
-                               pr[cc + 3] * (__uint_as_float(u[2 * e + 3]) - d4.w));
+          float g0 = __uint_as_float(u[2 * e]), g1 = __uint_as_float(u[2 * e + 1]);
+          float g2 = __uint_as_float(u[2 * e + 2]), g3 = __uint_as_float(u[2 * e + 3]);
+          if (DROPOUT) {  // dP = (dO V^T) o keep / (1 - p)
+            g0 = kept(cc) ? g0 * p.drop.keep_scale : 0.f;
+            g1 = kept(cc + 1) ? g1 * p.drop.keep_scale : 0.f;
+            g2 = kept(cc + 2) ? g2 * p.drop.keep_scale : 0.f;
+            g3 = kept(cc + 3) ? g3 * p.drop.keep_scale : 0.f;
+          }
+          w[e] = pack_bf16(pr[cc] * (g0 - d4.x), pr[cc + 1] * (g1 - d4.y));
+          w[e + 1] = pack_bf16(pr[cc + 2] * (g2 - d4.z), pr[cc + 3] * (g3 - d4.w));
         }
         // written over columns this thread has already read
         tmem_st16(tmem + lane_base + T_DP + cq + c * 16, w);
@@ -567,7 +606,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
 // ---------------------------------------------------------------------------
 // Kernel 2: dQ by an ordered walk over key blocks (deterministic mode)
 // ---------------------------------------------------------------------------
-template <int HD, bool ALIBI>
+template <int HD, bool ALIBI, bool DROPOUT>
 __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_constant__ BwdParams p) {
   using C = DqCfg<HD>;
   using namespace bwd_detail;
@@ -754,10 +793,21 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int cc = c * 32 + 2 * e;
-          w[e] = pack_bf16(pr[cc] * (__uint_as_float(u[2 * e]) - dval),
-                           pr[cc + 1] * (__uint_as_float(u[2 * e + 1]) - dval));
+        for (int e4 = 0; e4 < 8; ++e4) {
+          // dropout bytes of keys kv0 + c*32 + 4*e4 .. +3 for this row
+          uint32_t word = 0xFFFFFFFFu;
+          if (DROPOUT) word = dropout_word_row(p.drop, b, h, i, ((kv0 + c * 32) >> 2) + e4);
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int e = 2 * e4 + e2;
+            const int cc = c * 32 + 2 * e;
+            float g0 = __uint_as_float(u[2 * e]), g1 = __uint_as_float(u[2 * e + 1]);
+            if (DROPOUT) {
+              g0 = dropout_keep(word, 2 * e2, p.drop.threshold) ? g0 * p.drop.keep_scale : 0.f;
+              g1 = dropout_keep(word, 2 * e2 + 1, p.drop.threshold) ? g1 * p.drop.keep_scale : 0.f;
+            }
+            w[e] = pack_bf16(pr[cc] * (g0 - dval), pr[cc + 1] * (g1 - dval));
+          }
         }
         tmem_st16(tmem + lane_base + T_S + c * 16, w);   // dS (bf16) over S
       }

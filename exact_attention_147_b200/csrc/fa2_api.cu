@@ -58,9 +58,20 @@ fa2_status check_tensor(const void* p, const fa2_strides& s, fa2_dtype dtype) {
 fa2_status check_options(float softmax_scale, float dropout_p, const float* alibi) {
   if (std::isnan(softmax_scale) || std::isinf(softmax_scale)) return FA2_ERR_INVALID_ARG;
   if (std::isnan(dropout_p) || dropout_p < 0.f || dropout_p >= 1.f) return FA2_ERR_INVALID_ARG;
-  if (dropout_p != 0.f) return FA2_ERR_UNSUPPORTED;
+  // the byte threshold t = round(256 p) must leave something to keep
+  if (std::floor(double(dropout_p) * 256.0 + 0.5) > 255.0) return FA2_ERR_INVALID_ARG;
   if (alibi != nullptr && (reinterpret_cast<uintptr_t>(alibi) & 3u) != 0) return FA2_ERR_INVALID_ARG;
   return FA2_OK;
+}
+
+DropoutParams make_dropout(float dropout_p, unsigned long long seed) {
+  DropoutParams d;
+  const int t = int(std::floor(double(dropout_p) * 256.0 + 0.5));
+  d.seed_lo = uint32_t(seed & 0xFFFFFFFFull);
+  d.seed_hi = uint32_t(seed >> 32);
+  d.threshold = uint32_t(t);
+  d.keep_scale = float(256.0 / (256.0 - t));
+  return d;
 }
 
 #define FA2_TRY(expr)                 \
@@ -174,12 +185,16 @@ fa2_status launched(int n) {
   return FA2_OK;
 }
 
-std::atomic<uint64_t> g_smem_fwd128{0}, g_smem_fwd128a{0}, g_smem_fwd64{0}, g_smem_fwd64a{0};
+template <int HD>
+fa2_status dispatch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
+                              const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
+                              int causal_order, cudaStream_t st);
 
-template <int HD, bool ALIBI>
+template <int HD, bool ALIBI, bool DROPOUT>
 fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
                             const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
-                            int causal_order, cudaStream_t st, std::atomic<uint64_t>& mask) {
+                            int causal_order, cudaStream_t st) {
+  static std::atomic<uint64_t> mask{0};
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
   FA2_TRY(encode_bf16_4d(&p.tm_q, a.q, sq, a.B, a.N, a.H, HD, 128));
@@ -201,7 +216,8 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.heavy_first = causal_order;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.wait_ns = g_wait_ns.load();
-  auto kern = fa2_fwd_sm100_kernel<HD, ALIBI>;
+  p.drop = a.drop;
+  auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT>;
   constexpr int smem = FwdCfg<HD>::SMEM_BYTES;
   FA2_TRY(ensure_smem(kern, smem, dev, mask));
   // persistent grid: one CTA per SM (shared memory and TMEM allow one)
@@ -210,7 +226,7 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   return launched(1);
 }
 
-template <int HD, bool ALIBI>
+template <int HD, bool ALIBI, bool DROPOUT>
 fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
                             const fa2_strides& sv, const fa2_strides& sdo, const fa2_strides& sdq,
                             const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
@@ -240,6 +256,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.wait_ns = g_wait_ns.load();
+  p.drop = a.drop;
   const unsigned grid = unsigned(p.nblocks) * unsigned(a.H) * unsigned(a.B);
   constexpr int smem1 = BwdCfg<HD>::SMEM_BYTES;
   // Kernel 1 re-balances registers between its warpgroups; the shares add up
@@ -248,8 +265,8 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   // forever.  Refuse to launch otherwise.
   {
     cudaFuncAttributes fa;
-    auto k1c = deterministic ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false>
-                             : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true>;
+    auto k1c = deterministic ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT>
+                             : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT>;
     if (cudaFuncGetAttributes(&fa, k1c) != cudaSuccess) return FA2_ERR_CUDA;
     if (fa.numRegs < BwdCfg<HD>::REGS_AT_LAUNCH) return FA2_ERR_UNSUPPORTED;
   }
@@ -258,7 +275,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
     const unsigned zgrid = unsigned(std::min<long long>((n4 + 255) / 256, 148 * 16));
     zero_f32x4_kernel<<<zgrid, 256, 0, st>>>(reinterpret_cast<float4*>(a.dq_accum), n4);
     FA2_TRY(launched(1));
-    auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true>;
+    auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT>;
     FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv));
     k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
     FA2_TRY(launched(1));
@@ -267,15 +284,40 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
     dq_convert_kernel<HD><<<unsigned((rows + per_block - 1) / per_block), 256, 0, st>>>(a);
     return launched(1);
   }
-  auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false>;
+  auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT>;
   FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv_nodq));
   k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
   FA2_TRY(launched(1));
-  auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI>;
+  auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI, DROPOUT>;
   constexpr int smem2 = DqCfg<HD>::SMEM_BYTES;
   FA2_TRY(ensure_smem(k2, smem2, dev, mask_dq));
   k2<<<grid, DqCfg<HD>::THREADS, smem2, st>>>(p);
   return launched(1);
+}
+
+template <int HD>
+fa2_status dispatch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
+                              const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
+                              int causal_order, cudaStream_t st) {
+  if (a.alibi) {
+    return a.dropout ? launch_fwd_sm100<HD, true, true>(a, sq, sk, sv, so, dev, sm_count, causal_order, st)
+                     : launch_fwd_sm100<HD, true, false>(a, sq, sk, sv, so, dev, sm_count, causal_order, st);
+  }
+  return a.dropout ? launch_fwd_sm100<HD, false, true>(a, sq, sk, sv, so, dev, sm_count, causal_order, st)
+                   : launch_fwd_sm100<HD, false, false>(a, sq, sk, sv, so, dev, sm_count, causal_order, st);
+}
+
+template <int HD>
+fa2_status dispatch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
+                              const fa2_strides& sv, const fa2_strides& sdo, const fa2_strides& sdq,
+                              const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
+                              int dev, cudaStream_t st) {
+  if (a.alibi) {
+    return a.dropout ? launch_bwd_sm100<HD, true, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
+                     : launch_bwd_sm100<HD, true, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
+  }
+  return a.dropout ? launch_bwd_sm100<HD, false, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
+                   : launch_bwd_sm100<HD, false, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
 }
 
 }  // namespace
@@ -319,7 +361,8 @@ fa2_status fa2_device_status(int* code, int clear) {
 fa2_status fa2_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
                    int H, int d, fa2_dtype dtype, fa2_strides sq, fa2_strides sk, fa2_strides sv,
                    fa2_strides so, float softmax_scale, int causal, int window_left, int window_right,
-                   const float* alibi_slopes, float dropout_p, void* stream) {
+                   const float* alibi_slopes, float dropout_p, unsigned long long dropout_seed,
+                   void* stream) {
   FA2_TRY(check_shape(B, N, H, d, dtype));
   FA2_TRY(check_tensor(q, sq, dtype));
   FA2_TRY(check_tensor(k, sk, dtype));
@@ -338,6 +381,8 @@ fa2_status fa2_fwd(const void* q, const void* k, const void* v, void* o, float* 
   a.wl = window_left;
   a.wr = window_right;
   normalise_window(causal, &a.wl, &a.wr);
+  a.dropout = dropout_p != 0.f;
+  a.drop = make_dropout(dropout_p, dropout_seed);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   int dev;
@@ -352,12 +397,8 @@ fa2_status fa2_fwd(const void* q, const void* k, const void* v, void* o, float* 
   }
   if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;  // sm_100a kernels only
   const int heavy_first = (a.wr >= 0 || a.wl >= 0) ? 1 : 0;
-  if (d == 128) {
-    return alibi_slopes ? launch_fwd_sm100<128, true>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st, g_smem_fwd128a)
-                        : launch_fwd_sm100<128, false>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st, g_smem_fwd128);
-  }
-  return alibi_slopes ? launch_fwd_sm100<64, true>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st, g_smem_fwd64a)
-                      : launch_fwd_sm100<64, false>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st, g_smem_fwd64);
+  return d == 128 ? dispatch_fwd_sm100<128>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st)
+                  : dispatch_fwd_sm100<64>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st);
 }
 
 fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D, int B, int N, int H, int d,
@@ -402,7 +443,8 @@ fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout
                    fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides sdo,
                    fa2_strides sdq, fa2_strides sdk, fa2_strides sdv, float softmax_scale,
                    int causal, int window_left, int window_right, const float* alibi_slopes,
-                   float dropout_p, int deterministic, void* stream) {
+                   float dropout_p, unsigned long long dropout_seed, int deterministic,
+                   void* stream) {
   FA2_TRY(check_shape(B, N, H, d, dtype));
   FA2_TRY(check_tensor(q, sq, dtype));
   FA2_TRY(check_tensor(k, sk, dtype));
@@ -431,6 +473,8 @@ fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout
   a.wl = window_left;
   a.wr = window_right;
   normalise_window(causal, &a.wl, &a.wr);
+  a.dropout = dropout_p != 0.f;
+  a.drop = make_dropout(dropout_p, dropout_seed);
   int dev;
   DeviceInfo di;
   FA2_TRY(current_device(&dev, &di));
@@ -447,11 +491,8 @@ fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout
     return launched(2);
   }
   if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;
-  if (d == 128)
-    return alibi_slopes ? launch_bwd_sm100<128, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
-                        : launch_bwd_sm100<128, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
-  return alibi_slopes ? launch_bwd_sm100<64, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
-                      : launch_bwd_sm100<64, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
+  return d == 128 ? dispatch_bwd_sm100<128>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
+                  : dispatch_bwd_sm100<64>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -500,6 +541,7 @@ fa2_status fa2_bwd_noalloc(const void* q, const void* k, const void* v, const vo
   FA2_TRY(check_tensor(dv, sdv, dtype));
   if (lse == nullptr || !aligned16(lse) || D == nullptr || !aligned16(D)) return FA2_ERR_INVALID_ARG;
   FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
+  if (dropout_p != 0.f) return FA2_ERR_UNSUPPORTED;  // this entry point has no seed argument
   if ((unsigned long long)B * H * N * d > (unsigned long long)FA2_NOALLOC_MAX_DQ_FLOATS)
     return FA2_ERR_SCRATCH_LIMIT;
   int dev;
@@ -521,11 +563,8 @@ fa2_status fa2_bwd_noalloc(const void* q, const void* k, const void* v, const vo
   a.wr = window_right;
   normalise_window(causal, &a.wl, &a.wr);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128)
-    return alibi_slopes ? launch_bwd_sm100<128, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st)
-                        : launch_bwd_sm100<128, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st);
-  return alibi_slopes ? launch_bwd_sm100<64, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st)
-                      : launch_bwd_sm100<64, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st);
+  return d == 128 ? dispatch_bwd_sm100<128>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st)
+                  : dispatch_bwd_sm100<64>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st);
 }
 
 }  // extern "C"

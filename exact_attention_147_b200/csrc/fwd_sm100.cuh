@@ -50,6 +50,7 @@
 #include <math_constants.h>
 
 #include "attn_common.cuh"
+#include "philox.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fa2 {
@@ -67,6 +68,7 @@ struct FwdParams {
   int heavy_first;                     // order units longest-first (masks)
   float scale_log2;                    // softmax_scale * log2(e)
   unsigned long long wait_ns;          // bounded-wait limit
+  DropoutParams drop;                  // used by the DROPOUT instantiations
 };
 
 template <int HD>
@@ -141,7 +143,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-template <int HD, bool ALIBI>
+template <int HD, bool ALIBI, bool DROPOUT>
 __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<HD>;
   constexpr int BM = C::BM, BN = C::BN, NQT = C::NQT, SLOTS = C::SLOTS;
@@ -403,6 +405,15 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
           l3 += s[c + 3];
         }
         l_run = fmaf(l_run, alpha, (l0 + l1) + (l2 + l3));
+        if (DROPOUT) {  // l keeps the un-dropped sum; dropped probabilities leave P
+#pragma unroll
+          for (int c4 = 0; c4 < BN / 4; ++c4) {
+            const uint32_t word = dropout_word_row(p.drop, b, h, i, (kv0 >> 2) + c4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (!dropout_keep(word, e, p.drop.threshold)) s[4 * c4 + e] = 0.f;
+          }
+        }
         // P (bf16 pairs) over the first BN/2 columns of S.
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
@@ -434,7 +445,7 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv_l = l_run > 0.f ? (DROPOUT ? p.drop.keep_scale : 1.f) / l_run : 0.f;
       __nv_bfloat16* orow = p.o + b * p.so_b + (long long)i * p.so_n + h * p.so_h;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {

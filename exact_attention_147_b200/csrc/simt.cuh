@@ -71,10 +71,15 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(const AttnArgs a) {
     const float m_new = fmaxf(m, s);
     const float alpha = expf(m - m_new);   // 0 on the first visible key
     const float p = expf(s - m_new);
-    l = l * alpha + p;
+    l = l * alpha + p;                      // the un-dropped sum
+    float pk = p;
+    if (a.dropout) {
+      const uint32_t word = dropout_word_row(a.drop, b, h, i, j >> 2);
+      pk = dropout_keep(word, j & 3, a.drop.threshold) ? p * a.drop.keep_scale : 0.f;
+    }
     const T* vr = vb + j * a.sv.n;
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = fmaf(p, to_f(vr[lane + 32 * e]), acc[e] * alpha);
+    for (int e = 0; e < E; ++e) acc[e] = fmaf(pk, to_f(vr[lane + 32 * e]), acc[e] * alpha);
     m = m_new;
   }
   T* o = static_cast<T*>(a.o) + b * a.so.b + i * a.so.n + h * a.so.h;
@@ -121,12 +126,19 @@ __global__ void __launch_bounds__(128) simt_bwd_dkdv_kernel(const AttnArgs a) {
     }
     float s = warp_sum(ps) * a.scale;
     if (a.alibi) s -= slope * fabsf(float(i - j));
-    const float dp = warp_sum(pd);
+    float dp = warp_sum(pd);
     const float p = expf(s - lse[i]);
+    float pk = p;
+    if (a.dropout) {
+      const uint32_t word = dropout_word_row(a.drop, b, h, i, j >> 2);
+      const float km = dropout_keep(word, j & 3, a.drop.threshold) ? a.drop.keep_scale : 0.f;
+      pk = p * km;
+      dp *= km;
+    }
     const float ds = p * (dp - dvec[i]);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      dv[e] = fmaf(p, df[e], dv[e]);
+      dv[e] = fmaf(pk, df[e], dv[e]);
       dk[e] = fmaf(ds, qf[e], dk[e]);
     }
   }
@@ -174,8 +186,12 @@ __global__ void __launch_bounds__(128) simt_bwd_dq_kernel(const AttnArgs a) {
     }
     float s = warp_sum(ps) * a.scale;
     if (a.alibi) s -= slope * fabsf(float(i - j));
-    const float dp = warp_sum(pd);
+    float dp = warp_sum(pd);
     const float p = expf(s - lse_i);
+    if (a.dropout) {
+      const uint32_t word = dropout_word_row(a.drop, b, h, i, j >> 2);
+      dp *= dropout_keep(word, j & 3, a.drop.threshold) ? a.drop.keep_scale : 0.f;
+    }
     const float ds = p * (dp - d_i);
 #pragma unroll
     for (int e = 0; e < E; ++e) dq[e] = fmaf(ds, kf[e], dq[e]);

@@ -65,14 +65,15 @@ def load_library(path: str = LIB_PATH):
             "`python -m exact_attention_147_b200.build`")
     lib = ctypes.CDLL(path)
     vp, i, f, s = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, Strides
-    lib.fa2_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, s, s, s, s, f, i, i, i, vp, f, vp]
+    u64 = ctypes.c_uint64
+    lib.fa2_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, s, s, s, s, f, i, i, i, vp, f, u64, vp]
     lib.fa2_fwd.restype = i
     lib.fa2_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, i, s, s, vp]
     lib.fa2_bwd_preprocess.restype = i
     lib.fa2_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
     lib.fa2_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa2_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
-                            i, i, i, i, i, s, s, s, s, s, s, s, f, i, i, i, vp, f, i, vp]
+                            i, i, i, i, i, s, s, s, s, s, s, s, f, i, i, i, vp, f, u64, i, vp]
     lib.fa2_bwd.restype = i
     lib.fa2_strerror.argtypes = [i]
     lib.fa2_strerror.restype = ctypes.c_char_p
@@ -134,7 +135,7 @@ def _scale(softmax_scale):
 
 
 def fwd(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1),
-        alibi_slopes=None, dropout_p=0.0, out=None, lse=None, stream=None):
+        alibi_slopes=None, dropout_p=0.0, out=None, lse=None, stream=None, dropout_seed=0):
     """Forward pass; returns (out [B,N,H,d], lse [B,H,N] fp32)."""
     lib = load_library()
     B, N, H, d = q.shape
@@ -146,7 +147,7 @@ def fwd(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1),
     st = lib.fa2_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, N, H, d,
                      _dtype_code(q), _strides(q), _strides(k), _strides(v), _strides(out),
                      _scale(softmax_scale), c, wl, wr, _ptr(alibi_slopes),
-                     float(dropout_p), _stream(stream))
+                     float(dropout_p), int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, _stream(stream))
     _check(st, "fa2_fwd")
     return out, lse
 
@@ -170,7 +171,7 @@ def workspace_size(B, N, H, d, dtype, deterministic=False) -> int:
 
 def bwd(dout, q, k, v, lse, D, softmax_scale=None, causal=False, window_size=(-1, -1),
         alibi_slopes=None, dropout_p=0.0, deterministic=False, dq=None, dk=None, dv=None,
-        workspace=None, stream=None):
+        workspace=None, stream=None, dropout_seed=0):
     """Backward pass; returns (dq, dk, dv) shaped like q, k, v."""
     lib = load_library()
     B, N, H, d = q.shape
@@ -186,7 +187,8 @@ def bwd(dout, q, k, v, lse, D, softmax_scale=None, causal=False, window_size=(-1
                      _ptr(dk), _ptr(dv), _ptr(workspace), wbytes, B, N, H, d, _dtype_code(q),
                      _strides(q), _strides(k), _strides(v), _strides(dout), _strides(dq),
                      _strides(dk), _strides(dv), _scale(softmax_scale), c, wl, wr,
-                     _ptr(alibi_slopes), float(dropout_p), int(bool(deterministic)),
+                     _ptr(alibi_slopes), float(dropout_p),
+                     int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, int(bool(deterministic)),
                      _stream(stream))
     _check(st, "fa2_bwd")
     return dq, dk, dv
@@ -214,19 +216,22 @@ class _Fa2Function(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, dropout_p, softmax_scale, causal, window_size, alibi_slopes,
                 deterministic):
-        out, lse = fwd(q, k, v, softmax_scale, causal, window_size, alibi_slopes, dropout_p)
+        # a fresh mask per call, drawn from torch's default CPU generator
+        seed = int(torch.randint(0, 2**63 - 1, (1,)).item()) if dropout_p > 0 else 0
+        out, lse = fwd(q, k, v, softmax_scale, causal, window_size, alibi_slopes, dropout_p,
+                       dropout_seed=seed)
         ctx.save_for_backward(q, k, v, out, lse, alibi_slopes)
-        ctx.opts = (dropout_p, softmax_scale, causal, window_size, deterministic)
+        ctx.opts = (dropout_p, softmax_scale, causal, window_size, deterministic, seed)
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, out, lse, alibi_slopes = ctx.saved_tensors
-        dropout_p, softmax_scale, causal, window_size, deterministic = ctx.opts
+        dropout_p, softmax_scale, causal, window_size, deterministic, seed = ctx.opts
         dout = dout if dout.stride(-1) == 1 else dout.contiguous()
         D = bwd_preprocess(out, dout)
         dq, dk, dv = bwd(dout, q, k, v, lse, D, softmax_scale, causal, window_size,
-                         alibi_slopes, dropout_p, deterministic)
+                         alibi_slopes, dropout_p, deterministic, dropout_seed=seed)
         return dq, dk, dv, None, None, None, None, None, None
 
 

@@ -96,7 +96,20 @@ typedef struct {
  *                 ("window_size=(-1,-1)" is the default).
  *   alibi_slopes  NULL, or a device fp32 [H] array; adds -slope_h * |i - j|
  *                 to the scaled score (linear-bias attention).
- *   dropout_p     must be 0 (anything else returns FA2_ERR_UNSUPPORTED).
+ *   dropout_p     probability of zeroing each attention probability after
+ *                 the softmax, 0 <= dropout_p < 255.5/256; kept ones are
+ *                 scaled so the expected output is unchanged (see DROPOUT).
+ *   dropout_seed  64-bit seed of the dropout mask (ignored when
+ *                 dropout_p == 0).
+ *
+ * DROPOUT.  With t = round(256 * dropout_p), element (b, h, query i, key j)
+ * is kept iff its random byte is >= t, and kept probabilities are multiplied
+ * by 256 / (256 - t) (so the effective drop probability is t / 256).  The
+ * random byte is byte (j mod 4), least significant first, of output word
+ * (i mod 4) of Philox4x32-10 (Salmon et al., SC 2011) with counter
+ * (j / 4, i / 4, h, b) and key (dropout_seed mod 2^32, dropout_seed / 2^32).
+ * fa2_bwd with the same seed and dropout_p regenerates the same mask.  LSE
+ * is always the log-sum-exp of the un-dropped scores.
  *
  * A query row that sees no key (impossible with the masks above, since the
  * diagonal is always visible) gets O = 0 and lse = -inf.  The result is
@@ -106,7 +119,8 @@ fa2_status fa2_fwd(const void* q, const void* k, const void* v, void* o, float* 
                    int B, int N, int H, int d, fa2_dtype dtype,
                    fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides so,
                    float softmax_scale, int causal, int window_left, int window_right,
-                   const float* alibi_slopes, float dropout_p, void* stream);
+                   const float* alibi_slopes, float dropout_p, unsigned long long dropout_seed,
+                   void* stream);
 
 /*
  * Backward pre-processing: D[b, h, i] = sum_c dO[b, i, h, c] * O[b, i, h, c]
@@ -135,7 +149,8 @@ size_t fa2_bwd_workspace_size(int B, int N, int H, int d, fa2_dtype dtype, int d
  *   dq, dk, dv       [B, N, H, d] outputs (dtype) with strides sdq, sdk, sdv.
  *   workspace        device buffer of at least workspace_bytes >=
  *                    fa2_bwd_workspace_size(...) bytes, 256-byte aligned.
- *   softmax_scale, causal, window_left, window_right, alibi_slopes, dropout_p
+ *   softmax_scale, causal, window_left, window_right, alibi_slopes,
+ *   dropout_p, dropout_seed
  *                    exactly as passed to fa2_fwd.
  *   deterministic    0: dQ partial sums from different key blocks are added
  *                    with fp32 atomics (fast, order not fixed);
@@ -149,8 +164,8 @@ fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout
                    fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides sdo,
                    fa2_strides sdq, fa2_strides sdk, fa2_strides sdv,
                    float softmax_scale, int causal, int window_left, int window_right,
-                   const float* alibi_slopes, float dropout_p, int deterministic,
-                   void* stream);
+                   const float* alibi_slopes, float dropout_p, unsigned long long dropout_seed,
+                   int deterministic, void* stream);
 
 /*
  * fa2_bwd_noalloc: the bf16 backward pass without any caller-provided or
@@ -167,9 +182,10 @@ fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout
  * present on every GPU that loads the library until the process exits).
  * It calls no cudaMalloc, cudaFree or other allocating routine.
  *
- * Arguments and results are those of fa2_bwd with dtype FA2_BF16 and
- * deterministic = 0 (dQ partial sums added with fp32 atomics).  The caller
- * still provides q, k, v, dout, lse, D, dq, dk and dv.
+ * Arguments and results are those of fa2_bwd with dtype FA2_BF16,
+ * deterministic = 0 (dQ partial sums added with fp32 reductions) and no
+ * dropout (dropout_p != 0 returns FA2_ERR_UNSUPPORTED).  The caller still
+ * provides q, k, v, dout, lse, D, dq, dk and dv.
  *
  *   Limit:   B * H * N * d must not exceed FA2_NOALLOC_MAX_DQ_FLOATS;
  *            larger problems return FA2_ERR_SCRATCH_LIMIT and launch

@@ -53,27 +53,25 @@ def call_fwd(lib, **kw):
     a.update(kw)
     return lib.fa2_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["N"], a["H"], a["d"],
                        a["dtype"], a["s"], a["s"], a["s"], a["s"], a["scale"], a["causal"],
-                       a["wl"], a["wr"], a["alibi"], a["dropout"], None)
+                       a["wl"], a["wr"], a["alibi"], a["dropout"], 0, None)
 
 
 @pytest.mark.parametrize("bad", [
     dict(q=None), dict(k=None), dict(lse=None), dict(d=96), dict(d=0), dict(N=0), dict(B=0),
     dict(H=-1), dict(dtype=7), dict(q=ctypes.c_void_p(0x100008)),
     dict(s=F.Strides(8, 12, 128)), dict(s=F.Strides(0, 128, 128)), dict(scale=float("nan")),
-    dict(dropout=float("nan")), dict(dropout=1.5), dict(alibi=ctypes.c_void_p(0x100002)),
+    dict(dropout=float("nan")), dict(dropout=1.5), dict(dropout=0.999), dict(dropout=-0.1),
+    dict(alibi=ctypes.c_void_p(0x100002)),
     dict(o=P),  # output aliases an input
 ])
 def test_fwd_rejects_invalid(lib, bad):
     assert call_fwd(lib, **bad) == F.FA2_ERR_INVALID_ARG
 
 
-def test_fwd_dropout_unsupported(lib):
-    assert call_fwd(lib, dropout=0.1) == F.FA2_ERR_UNSUPPORTED
-
-
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
 def test_valid_call_without_device_is_cuda_error(lib):
     assert call_fwd(lib) == F.FA2_ERR_CUDA
+    assert call_fwd(lib, dropout=0.25) == F.FA2_ERR_CUDA   # a valid dropout probability
 
 
 def test_preprocess_and_bwd_reject_invalid(lib):
@@ -87,14 +85,14 @@ def test_preprocess_and_bwd_reject_invalid(lib):
     st = lib.fa2_bwd(P, P, P, P, P, P, ctypes.c_void_p(0x300000), ctypes.c_void_p(0x400000),
                      ctypes.c_void_p(0x500000), ctypes.c_void_p(0x600000), need - 1,
                      1, 256, 2, 128, F.FA2_BF16, s, s, s, s, s, s, s, 0.0, 0, -1, -1, None,
-                     0.0, 0, None)
+                     0.0, 0, 0, None)
     assert st == F.FA2_ERR_INVALID_ARG
-    # dropout
+    # dropout probability whose byte threshold would keep nothing
     st = lib.fa2_bwd(P, P, P, P, P, P, ctypes.c_void_p(0x300000), ctypes.c_void_p(0x400000),
                      ctypes.c_void_p(0x500000), ctypes.c_void_p(0x600000), need,
                      1, 256, 2, 128, F.FA2_BF16, s, s, s, s, s, s, s, 0.0, 0, -1, -1, None,
-                     0.2, 0, None)
-    assert st == F.FA2_ERR_UNSUPPORTED
+                     0.999, 0, 0, None)
+    assert st == F.FA2_ERR_INVALID_ARG
 
 
 def test_workspace_size(lib):

@@ -1,0 +1,137 @@
+"""Dropout parity: libfa2's dropout mask and gradients against the oracle.
+
+The mask itself is compared bit for bit: with q = 0 every visible key gets
+the same probability, so a one-hot value row makes each output element
+count the kept keys that land on it (forward), and a one-hot dO row does the
+same for dV (backward key-row kernel).  Outputs and gradients are then
+compared with the fp64 oracle, which draws the same mask with its own
+Philox4x32-10.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from exact_attention_147_b200 import fa2 as F
+from exact_attention_147_b200 import workloads as W
+from oracle import attention as oa
+from oracle import philox
+from tests.helpers import check_fwd, check_grad, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def onehot_rows(n, d, dtype):
+    v = torch.zeros(n, d)
+    v[torch.arange(n), torch.arange(n) % d] = 1.0
+    return v.to(dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("p,seed", [(0.5, 11), (0.1, 2**40 + 7)])
+def test_mask_bits_forward_and_backward(dtype, p, seed):
+    B, N, H, d = 2, 256, 3, 128
+    q = torch.zeros(B, N, H, d, dtype=dtype, device="cuda")
+    g = torch.Generator().manual_seed(3)
+    k = torch.randn(B, N, H, d, generator=g).to(dtype).cuda()
+    base = onehot_rows(N, d, dtype)                      # key j -> column j mod d
+    v = base[None, :, None, :].expand(B, N, H, d).contiguous().cuda()
+    out, lse = F.fwd(q, k, v, dropout_p=p, dropout_seed=seed)
+    do = base[None, :, None, :].expand(B, N, H, d).contiguous().cuda()  # query i -> column i mod d
+    D = F.bwd_preprocess(out, do)
+    dq, dk, dv = F.bwd(do, q, k, v, lse, D, dropout_p=p, dropout_seed=seed)
+    torch.cuda.synchronize()
+    assert F.device_status() == 0
+    ks = philox.keep_scale(p)
+    for b in range(B):
+        for h in range(H):
+            keep = philox.keep_mask(b, h, np.arange(N), N, p, seed).astype(np.float64)
+            # forward: O[i, c] = ks / N * (# kept keys j with j mod d == c)
+            cnt_f = keep.reshape(N, N // d, d).sum(axis=1)
+            got_f = np.rint(f64(out[b, :, h]) * N / ks)
+            assert np.array_equal(got_f, cnt_f), f"forward mask mismatch b={b} h={h}"
+            # backward: dV[j, c] = ks / N * (# kept queries i with i mod d == c)
+            cnt_b = keep.T.reshape(N, N // d, d).sum(axis=1)
+            got_b = np.rint(f64(dv[b, :, h]) * N / ks)
+            assert np.array_equal(got_b, cnt_b), f"backward mask mismatch b={b} h={h}"
+
+
+CASES = [
+    W.Workload("drop-n300-d128", B=2, N=300, H=2, d=128, seed=51),
+    W.Workload("drop-n300-d128-causal", B=1, N=300, H=2, d=128, causal=True, seed=52),
+    W.Workload("drop-n513-d64", B=1, N=513, H=2, d=64, seed=53),
+    W.Workload("drop-alibi-window", B=1, N=400, H=2, d=128, causal=True, alibi=True,
+               window_left=150, window_right=0, seed=54),
+    W.Workload("drop-det", B=1, N=384, H=2, d=128, causal=True, deterministic=True, seed=55),
+    W.Workload("drop-fp32", B=1, N=256, H=2, d=64, dtype=torch.float32, causal=True, seed=56,
+               scale=1.0 / 8.0),
+]
+
+
+@pytest.mark.parametrize("p", [0.1, 0.5])
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_dropout_parity(w, p):
+    seed = 1234 + w.seed
+    q, k, v, do = W.make_inputs(w, "cuda")
+    slopes = w.alibi_slopes()
+    sl = None if slopes is None else slopes.cuda()
+    win = (w.window_left, w.window_right)
+    out, lse = F.fwd(q, k, v, w.scale, w.causal, win, sl, p, dropout_seed=seed)
+    D = F.bwd_preprocess(out, do)
+    dq, dk, dv = F.bwd(do, q, k, v, lse, D, w.scale, w.causal, win, sl, p, w.deterministic,
+                       dropout_seed=seed)
+    torch.cuda.synchronize()
+    assert F.device_status() == 0
+    ks = philox.keep_scale(p)
+    for b in range(w.B):
+        for h in range(w.H):
+            keep = philox.keep_mask(b, h, np.arange(w.N), w.N, p, seed)
+            slope = None if slopes is None else float(slopes[h])
+            args = (f64(q[b, :, h]), f64(k[b, :, h]), f64(v[b, :, h]))
+            o_ref, l_ref = oa.head_forward(*args, w.softmax_scale, w.causal, w.window_left,
+                                           w.window_right, slope, keep=keep, keep_scale=ks)
+            # the dropped output has a larger range; bf16 rounding scales with it
+            o_max = None
+            if w.dtype == torch.bfloat16:
+                o_max = max(1e-2, ks * float(v[b, :, h].abs().max()) / 256.0)
+            check_fwd(f64(out[b, :, h]), f64(lse[b, h]), o_ref, l_ref, w.dtype,
+                      f"{w.name} p={p} ({b},{h})", o_max=o_max)
+            rdq, rdk, rdv, _ = oa.head_backward(*args, f64(do[b, :, h]), w.softmax_scale,
+                                                w.causal, w.window_left, w.window_right, slope,
+                                                keep=keep, keep_scale=ks)
+            tag = f"{w.name} p={p} ({b},{h})"
+            check_grad(f64(dq[b, :, h]), rdq, w.dtype, tag + " dq")
+            check_grad(f64(dk[b, :, h]), rdk, w.dtype, tag + " dk")
+            check_grad(f64(dv[b, :, h]), rdv, w.dtype, tag + " dv")
+
+
+def test_dropout_mid_sampled_heads():
+    w = W.mid(False)
+    p, seed = 0.1, 99
+    q, k, v, do = W.make_inputs(w, "cuda")
+    out, lse = F.fwd(q, k, v, dropout_p=p, dropout_seed=seed)
+    D = F.bwd_preprocess(out, do)
+    dq, dk, dv = F.bwd(do, q, k, v, lse, D, dropout_p=p, dropout_seed=seed)
+    torch.cuda.synchronize()
+    ks = philox.keep_scale(p)
+    for b, h in [(0, 0), (7, 15)]:
+        keep = philox.keep_mask(b, h, np.arange(w.N), w.N, p, seed)
+        args = (f64(q[b, :, h]), f64(k[b, :, h]), f64(v[b, :, h]))
+        o_ref, l_ref = oa.head_forward(*args, w.softmax_scale, keep=keep, keep_scale=ks)
+        check_fwd(f64(out[b, :, h]), f64(lse[b, h]), o_ref, l_ref, w.dtype, f"mid ({b},{h})")
+        rdq, rdk, rdv, _ = oa.head_backward(*args, f64(do[b, :, h]), w.softmax_scale,
+                                            keep=keep, keep_scale=ks)
+        check_grad(f64(dq[b, :, h]), rdq, w.dtype, "mid dq")
+        check_grad(f64(dk[b, :, h]), rdk, w.dtype, "mid dk")
+        check_grad(f64(dv[b, :, h]), rdv, w.dtype, "mid dv")
+
+
+def test_autograd_draws_fresh_masks():
+    w = W.Workload("ag-drop", B=1, N=256, H=2, d=128, seed=61)
+    q, k, v, do = W.make_inputs(w, "cuda")
+    o1 = F.flash_attention_v2(q, k, v, dropout_p=0.3)
+    o2 = F.flash_attention_v2(q, k, v, dropout_p=0.3)
+    assert not torch.equal(o1, o2)
+    qg = q.clone().requires_grad_(True)
+    F.flash_attention_v2(qg, k, v, dropout_p=0.3).backward(do)
+    assert torch.isfinite(qg.grad).all()
