@@ -390,12 +390,45 @@ def run_gpu(args):
             line["cpu_baseline"] = {"error": str(ex)}
     if world == 1 and not args.no_by_n:
         line["by_n"] = run_sweep(F, W, args, full=args.sweep)
+        line["dropout"] = run_dropout(F, W)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def run_dropout(F, W, p=0.1):
+    """The bench workload with attention dropout (fwd and bwd timed apart)."""
+    import torch
+    w = W.mid(False)
+    q, k, v, do = W.make_inputs(w, "cuda")
+    out, lse = F.fwd(q, k, v, dropout_p=p, dropout_seed=5)
+    D = F.bwd_preprocess(out, do)
+    dq, dk, dv = F.bwd(do, q, k, v, lse, D, dropout_p=p, dropout_seed=5)
+    ws = torch.empty(F.workspace_size(w.B, w.N, w.H, w.d, torch.bfloat16), dtype=torch.uint8,
+                     device="cuda")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for _ in range(3):
+        F.fwd(q, k, v, dropout_p=p, dropout_seed=5, out=out, lse=lse)
+        F.bwd(do, q, k, v, lse, D, dropout_p=p, dropout_seed=5, dq=dq, dk=dk, dv=dv, workspace=ws)
+    torch.cuda.synchronize()
+    reps = 10
+    ev[0].record()
+    for _ in range(reps):
+        F.fwd(q, k, v, dropout_p=p, dropout_seed=5, out=out, lse=lse)
+    ev[1].record()
+    for _ in range(reps):
+        F.bwd(do, q, k, v, lse, D, dropout_p=p, dropout_seed=5, dq=dq, dk=dk, dv=dv, workspace=ws)
+    ev[2].record()
+    torch.cuda.synchronize()
+    ff = flops_fwd(w.B, w.H, w.N, w.d)
+    tf = ev[0].elapsed_time(ev[1]) / reps
+    tb = ev[1].elapsed_time(ev[2]) / reps
+    return {"dropout_p": p, "workload": "B=8 H=16 N=2048 d=128", "fwd_ms": round(tf, 4),
+            "fwd_tflops": round(ff / (tf * 1e-3) / 1e12, 1), "bwd_ms": round(tb, 4),
+            "bwd_tflops": round(2.5 * ff / (tb * 1e-3) / 1e12, 1)}
 
 
 def run_sweep(F, W, args, full=False):
