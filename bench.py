@@ -391,6 +391,7 @@ def run_gpu(args):
     if world == 1 and not args.no_by_n:
         line["by_n"] = run_sweep(F, W, args, full=args.sweep)
         line["dropout"] = run_dropout(F, W)
+        line["packed"] = run_packed(F, W)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -429,6 +430,73 @@ def run_dropout(F, W, p=0.1):
     return {"dropout_p": p, "workload": "B=8 H=16 N=2048 d=128", "fwd_ms": round(tf, 4),
             "fwd_tflops": round(ff / (tf * 1e-3) / 1e12, 1), "bwd_ms": round(tb, 4),
             "bwd_tflops": round(2.5 * ff / (tb * 1e-3) / 1e12, 1)}
+
+
+def _time_pair(fwd_call, bwd_call, reps=10):
+    """Mean ms of fwd_call and of bwd_call (CUDA events on the current stream)."""
+    import torch
+    for _ in range(3):
+        fwd_call()
+        bwd_call()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    for _ in range(reps):
+        fwd_call()
+    ev[1].record()
+    for _ in range(reps):
+        bwd_call()
+    ev[2].record()
+    torch.cuda.synchronize()
+    return ev[0].elapsed_time(ev[1]) / reps, ev[1].elapsed_time(ev[2]) / reps
+
+
+def run_packed(F, W):
+    """A packed batch of mixed-length sequences (32768 tokens, lengths 128 to
+    4096) against the same sequences padded to the longest one.  TFLOP/s
+    count the useful work, sum over sequences of 4 L^2 d H (halved when
+    causal); the padded times are for the same useful work."""
+    import torch
+    res = []
+    for causal in (False, True):
+        w = W.packed_mix(causal)
+        q, k, v, do = W.make_inputs(w, "cuda")
+        cu = w.cu_seqlens("cuda")
+        out, lse = F.fwd_varlen(q, k, v, cu, w.N, causal=causal)
+        D = F.bwd_preprocess(out, do)
+        dq, dk, dv = F.bwd_varlen(do, q, k, v, lse, D, cu, w.N, causal=causal)
+        ws = torch.empty(F.workspace_size(1, w.total, w.H, w.d, torch.bfloat16),
+                         dtype=torch.uint8, device="cuda")
+        tf, tb = _time_pair(
+            lambda: F.fwd_varlen(q, k, v, cu, w.N, causal=causal, out=out, lse=lse),
+            lambda: F.bwd_varlen(do, q, k, v, lse, D, cu, w.N, causal=causal, dq=dq, dk=dk,
+                                 dv=dv, workspace=ws))
+        ff = sum(flops_fwd(1, w.H, n, w.d, causal) for n in w.lengths)
+        # the same sequences padded to the longest, as one padded call
+        B, N = w.B, w.N
+        qp, kp, vp, dop = (torch.zeros((B, N, w.H, w.d), dtype=t.dtype, device="cuda")
+                           for t in (q, k, v, do))
+        for b, n in enumerate(w.lengths):
+            s = int(sum(w.lengths[:b]))
+            for tp, t in ((qp, q), (kp, k), (vp, v), (dop, do)):
+                tp[b, :n] = t[s:s + n]
+        op_, lp = F.fwd(qp, kp, vp, causal=causal)
+        Dp = F.bwd_preprocess(op_, dop)
+        gp = F.bwd(dop, qp, kp, vp, lp, Dp, causal=causal)
+        wsp = torch.empty(F.workspace_size(B, N, w.H, w.d, torch.bfloat16), dtype=torch.uint8,
+                          device="cuda")
+        pf, pb = _time_pair(
+            lambda: F.fwd(qp, kp, vp, causal=causal, out=op_, lse=lp),
+            lambda: F.bwd(dop, qp, kp, vp, lp, Dp, causal=causal, dq=gp[0], dk=gp[1], dv=gp[2],
+                          workspace=wsp))
+        res.append({"workload": w.name, "sequences": w.B, "max_len": w.N, "tokens": w.total,
+                    "causal": causal, "fwd_ms": round(tf, 4),
+                    "fwd_tflops": round(ff / (tf * 1e-3) / 1e12, 1), "bwd_ms": round(tb, 4),
+                    "bwd_tflops": round(2.5 * ff / (tb * 1e-3) / 1e12, 1),
+                    "padded_fwd_ms": round(pf, 4), "padded_bwd_ms": round(pb, 4)})
+        del q, k, v, do, out, lse, D, dq, dk, dv, ws, qp, kp, vp, dop, op_, lp, Dp, gp, wsp
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_sweep(F, W, args, full=False):

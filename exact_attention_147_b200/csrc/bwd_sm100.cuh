@@ -45,14 +45,19 @@
 namespace fa2 {
 
 struct BwdParams {
-  CUtensorMap tm_q, tm_k, tm_v, tm_do;   // inputs, box {64,1,128,1}
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;   // inputs, box {64,1,128,1} (packed: [1,total,H,d])
   CUtensorMap tm_dq, tm_dk, tm_dv;       // outputs (bf16), same boxes
-  CUtensorMap tm_dqacc;                  // fp32 [B*H, N, d] accumulator, box {32,32,1}
-  const float* lse;                      // [B,H,N]
-  const float* dvec;                     // [B,H,N]
-  float* dq_accum;                       // [B,H,N,d] fp32 (kernel 1 with dQ)
+  CUtensorMap tm_dqacc;                  // fp32 [B*H, N, d] / [H, total, d] accumulator, box {32,32,1}
+  __nv_bfloat16 *dq, *dk, *dv;           // the outputs again, for row-wise stores of
+  Strides sdq, sdk, sdv;                 // tiles that end past a packed sequence
+  const float* lse;                      // [B,H,N] / [H,total]
+  const float* dvec;                     // same layout
+  float* dq_accum;                       // fp32 accumulator (kernel 1 with dQ)
   const float* alibi;                    // [H] or null
-  int N, H, B;
+  const int* cu_seqlens;                 // [B+1] sequence offsets (packed) or null (padded)
+  int total;                             // packed: tensor rows
+  int stat_rows;                         // rows per (batch, head) of lse / D: N or total
+  int N, H, B;                           // N: the (longest) sequence length
   int wl, wr;
   int nblocks;                           // ceil(N / 128)
   int heavy_first;
@@ -129,6 +134,18 @@ __device__ __forceinline__ void st_sw128_row32(uint8_t* tile, int row, int col0,
     *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
   }
 }
+
+// Writes the same 16 words straight to row `row` of a global bf16 tensor
+// (columns col0 .. col0 + 31): the output path of tiles whose last rows
+// belong to the next sequence of a packed batch, which a TMA store of the
+// whole tile would overwrite.
+__device__ __forceinline__ void st_global_row32(__nv_bfloat16* base, const Strides& s, const SeqView& v,
+                                                int row, int h, int col0, const uint32_t (&w)[16]) {
+  __nv_bfloat16* dst = row_ptr<__nv_bfloat16>(base, s, v, row, h) + col0;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4)
+    reinterpret_cast<uint4*>(dst)[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+}
 }  // namespace bwd_detail
 
 // ---------------------------------------------------------------------------
@@ -147,7 +164,7 @@ __device__ __forceinline__ void st_sw128_row32(uint8_t* tile, int row, int col0,
 // adds it into the fp32 accumulator with TMA bulk reductions, which go
 // through the TMA unit rather than the load/store queues.
 // ---------------------------------------------------------------------------
-template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT>
+template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT, bool PACKED>
 __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<HD>;
   using namespace bwd_detail;
@@ -195,13 +212,17 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
     hb = int(blockIdx.x / p.nblocks);
   }
   const int h = hb % p.H, b = hb / p.H;
-  const int k0 = kb * 128;
-  const int k_last = min(p.N - 1, k0 + 127);
+  const SeqView sv = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};
+  const int len = sv.len;
+  const int k0 = kb * 128;        // local key row of this block
+  if (k0 >= len) return;          // past the end of a shorter packed sequence: no work
+  const int k_last = min(len - 1, k0 + 127);
   const int i_lo = p.wr >= 0 ? max(0, k0 - p.wr) : 0;
-  const int i_hi = p.wl >= 0 ? min(p.N - 1, k_last + p.wl) : p.N - 1;
+  const int i_hi = p.wl >= 0 ? min(len - 1, k_last + p.wl) : len - 1;
   const int qb_begin = i_lo / 128;
   const int nq = i_hi / 128 - qb_begin + 1;
-  const size_t head_off = (size_t(b) * p.H + h) * p.N;
+  const size_t head_off = (size_t(sv.bt) * p.H + h) * (PACKED ? p.stat_rows : p.N) + sv.row0;
+  const int trow = sv.row0;       // tensor row of local row 0
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -230,8 +251,8 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       if (lane == 0) {
         bar_arrive_expect_tx(kv_full, 2 * C::TILE);
         for (int c = 0; c < NCH; ++c) {
-          tma_load_4d(smem_u32(sK + c * 16384), &p.tm_k, kv_full, c * 64, h, k0, b);
-          tma_load_4d(smem_u32(sV + c * 16384), &p.tm_v, kv_full, c * 64, h, k0, b);
+          tma_load_4d(smem_u32(sK + c * 16384), &p.tm_k, kv_full, c * 64, h, trow + k0, sv.bt);
+          tma_load_4d(smem_u32(sV + c * 16384), &p.tm_v, kv_full, c * 64, h, trow + k0, sv.bt);
         }
       }
       int issued_q = 0, issued_do = 0;
@@ -239,7 +260,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       for (int it = 0; it < nq && ok; ++it) {
         const int i0 = (qb_begin + it) * 128;
         const int sq = it % QS;
-        // log2-scaled LSE and D of this query block, +inf / 0 past N; loaded
+        // log2-scaled LSE and D of this query block, +inf / 0 past the end; loaded
         // before waiting for the slot so the latency overlaps the wait
         float l2v[4], dvv[4];
 #pragma unroll
@@ -247,7 +268,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           const int i = i0 + lane + 32 * e;
           l2v[e] = CUDART_INF_F;
           dvv[e] = 0.f;
-          if (i < p.N) {
+          if (i < len) {
             const float l = p.lse[head_off + i];
             l2v[e] = l == -CUDART_INF_F ? CUDART_INF_F : l * LOG2E;
             dvv[e] = p.dvec[head_off + i];
@@ -267,7 +288,8 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         if (lane == 0) {
           bar_arrive_expect_tx(q_full(sq), C::TILE);
           for (int c = 0; c < NCH; ++c)
-            tma_load_4d(smem_u32(sQ + sq * C::TILE + c * 16384), &p.tm_q, q_full(sq), c * 64, h, i0, b);
+            tma_load_4d(smem_u32(sQ + sq * C::TILE + c * 16384), &p.tm_q, q_full(sq), c * 64, h, trow + i0,
+                        sv.bt);
         }
         ++issued_q;
         const int sd = it % DS;
@@ -277,8 +299,8 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         if (lane == 0) {
           bar_arrive_expect_tx(do_full(sd), C::TILE);
           for (int c = 0; c < NCH; ++c)
-            tma_load_4d(smem_u32(sDO + sd * C::TILE + c * 16384), &p.tm_do, do_full(sd), c * 64, h, i0,
-                        b);
+            tma_load_4d(smem_u32(sDO + sd * C::TILE + c * 16384), &p.tm_do, do_full(sd), c * 64, h,
+                        trow + i0, sv.bt);
         }
         ++issued_do;
       }
@@ -380,8 +402,8 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
     const int j = k0 + r;
     const int cq = 64 * wg;  // this warpgroup's query columns [cq, cq + 64)
     int lo_q = p.wr >= 0 ? max(0, j - p.wr) : 0;
-    int hi_q = p.wl >= 0 ? min(p.N - 1, j + p.wl) : p.N - 1;
-    if (j >= p.N) {
+    int hi_q = p.wl >= 0 ? min(len - 1, j + p.wl) : len - 1;
+    if (j >= len) {
       lo_q = 1;
       hi_q = 0;
     }
@@ -515,6 +537,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
     if (ok) ok = wait_bar(acc_full, 0, ab, p.wait_ns, SITE_BCOMP + 2);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
+    // A whole tile leaves by TMA store; a tile whose last rows belong to the
+    // next packed sequence is written row by row instead.  (The sequence's
+    // rows are looked up again here rather than kept live through the loop.)
+    const SeqView so = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};
+    const bool tile_store = !PACKED || k0 + 128 <= so.len;
     if (ok) {
       // this warpgroup's half of the d columns of dV and dK -> bf16 -> the
       // V and K tiles (free now) -> TMA store
@@ -526,21 +553,23 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e) w[e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
-        st_sw128_row32(sV, r, col, w);
+        if (tile_store) st_sw128_row32(sV, r, col, w);
+        else if (j < so.len) st_global_row32(p.dv, p.sdv, so, j, h, col, w);
         tmem_ld32(tmem + lane_base + T_DK + col, u);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16(__uint_as_float(u[2 * e]) * p.scale, __uint_as_float(u[2 * e + 1]) * p.scale);
-        st_sw128_row32(sK, r, col, w);
+        if (tile_store) st_sw128_row32(sK, r, col, w);
+        else if (j < so.len) st_global_row32(p.dk, p.sdk, so, j, h, col, w);
       }
     }
     fence_proxy_async_smem();
     named_bar_sync(1, 256);
-    if (ok && threadIdx.x == 0) {
+    if (ok && tile_store && threadIdx.x == 0) {
       for (int c = 0; c < NCH; ++c) {
-        tma_store_4d(&p.tm_dv, smem_u32(sV + c * 16384), c * 64, h, k0, b);
-        tma_store_4d(&p.tm_dk, smem_u32(sK + c * 16384), c * 64, h, k0, b);
+        tma_store_4d(&p.tm_dv, smem_u32(sV + c * 16384), c * 64, h, so.row0 + k0, so.bt);
+        tma_store_4d(&p.tm_dk, smem_u32(sK + c * 16384), c * 64, h, so.row0 + k0, so.bt);
       }
       bulk_commit();
       bulk_wait_all();
@@ -551,7 +580,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       // ---------------------------------------------------------- dQ drain (query rows)
       const int q = (warp % 4) * 32 + lane;
       const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
-      const int bh = b * p.H + h;
+      const int bh = sv.bt * p.H + h;
       for (int it = 0; it < nq; ++it) {
         const int i0 = (qb_begin + it) * 128;
         bool ok = wait_bar(dq_full, it & 1, ab, p.wait_ns, SITE_BRED);
@@ -577,7 +606,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           __syncwarp();
           if (lane == 0) {
             tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sStg + (chunk & 1) * 16384 + wq * 4096), chunk * 32,
-                              i0 + wq * 32, bh);
+                              trow + i0 + wq * 32, bh);
             bulk_commit();
           }
         };
@@ -606,7 +635,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
 // ---------------------------------------------------------------------------
 // Kernel 2: dQ by an ordered walk over key blocks (deterministic mode)
 // ---------------------------------------------------------------------------
-template <int HD, bool ALIBI, bool DROPOUT>
+template <int HD, bool ALIBI, bool DROPOUT, bool PACKED>
 __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_constant__ BwdParams p) {
   using C = DqCfg<HD>;
   using namespace bwd_detail;
@@ -643,13 +672,17 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
     hb = int(blockIdx.x / p.nblocks);
   }
   const int h = hb % p.H, b = hb / p.H;
-  const int i0 = qb * 128;
-  const int i_last = min(p.N - 1, i0 + 127);
+  const SeqView sv = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};
+  const int len = sv.len;
+  const int i0 = qb * 128;        // local query row of this block
+  if (i0 >= len) return;          // past the end of a shorter packed sequence: no work
+  const int i_last = min(len - 1, i0 + 127);
   const int kv_lo = p.wl >= 0 ? max(0, i0 - p.wl) : 0;
-  const int kv_hi = p.wr >= 0 ? min(p.N - 1, i_last + p.wr) : p.N - 1;
+  const int kv_hi = p.wr >= 0 ? min(len - 1, i_last + p.wr) : len - 1;
   const int kb_begin = kv_lo / 128;
   const int nk = kv_hi / 128 - kb_begin + 1;
-  const size_t head_off = (size_t(b) * p.H + h) * p.N;
+  const size_t head_off = (size_t(sv.bt) * p.H + h) * (PACKED ? p.stat_rows : p.N) + sv.row0;
+  const int trow = sv.row0;       // tensor row of local row 0
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -673,13 +706,13 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
     if (lane == 0) {
       bar_arrive_expect_tx(qd_full, 2 * C::TILE);
       for (int c = 0; c < NCH; ++c) {
-        tma_load_4d(smem_u32(sQ + c * 16384), &p.tm_q, qd_full, c * 64, h, i0, b);
-        tma_load_4d(smem_u32(sDO + c * 16384), &p.tm_do, qd_full, c * 64, h, i0, b);
+        tma_load_4d(smem_u32(sQ + c * 16384), &p.tm_q, qd_full, c * 64, h, trow + i0, sv.bt);
+        tma_load_4d(smem_u32(sDO + c * 16384), &p.tm_do, qd_full, c * 64, h, trow + i0, sv.bt);
       }
       int n = 0;
       bool ok = true;
       for (int it = 0; it < nk && ok; ++it) {
-        const int kv0 = (kb_begin + it) * 128;
+        const int kv0 = trow + (kb_begin + it) * 128;
         for (int which = 0; which < 2; ++which, ++n) {
           const int s = n % SLOTS;
           if (!wait_bar(slot_empty(s), ((n / SLOTS) & 1) ^ 1, ab, p.wait_ns, SITE_QPROD)) {
@@ -689,7 +722,7 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
           bar_arrive_expect_tx(slot_full(s), C::TILE);
           const CUtensorMap* tm = which == 0 ? &p.tm_k : &p.tm_v;
           for (int c = 0; c < NCH; ++c)
-            tma_load_4d(smem_u32(sKV + s * C::TILE + c * 16384), tm, slot_full(s), c * 64, h, kv0, b);
+            tma_load_4d(smem_u32(sKV + s * C::TILE + c * 16384), tm, slot_full(s), c * 64, h, kv0, sv.bt);
         }
       }
       drain_wait(qd_full, 0, p.wait_ns);
@@ -742,11 +775,11 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
     const int r = warp * 32 + lane;
     const int i = i0 + r;
     const int lo = p.wl >= 0 ? max(0, i - p.wl) : 0;
-    const int hi = i >= p.N ? -1 : (p.wr >= 0 ? min(p.N - 1, i + p.wr) : p.N - 1);
+    const int hi = i >= len ? -1 : (p.wr >= 0 ? min(len - 1, i + p.wr) : len - 1);
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
     const float C2 = p.scale_log2;
     float lse2 = CUDART_INF_F, dval = 0.f, slope2 = 0.f;
-    if (i < p.N) {
+    if (i < len) {
       const float l = p.lse[head_off + i];
       lse2 = l == -CUDART_INF_F ? CUDART_INF_F : l * LOG2E;
       dval = p.dvec[head_off + i];
@@ -818,6 +851,8 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
     if (ok) ok = wait_bar(acc_full, 0, ab, p.wait_ns, SITE_QCOMP + 2);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
+    const SeqView so = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};
+    const bool tile_store = !PACKED || i0 + 128 <= so.len;
     if (ok) {
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
@@ -827,13 +862,15 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16(__uint_as_float(u[2 * e]) * p.scale, __uint_as_float(u[2 * e + 1]) * p.scale);
-        st_sw128_row32(sQ, r, c * 32, w);   // Q tile is free once every MMA is done
+        if (tile_store) st_sw128_row32(sQ, r, c * 32, w);   // Q tile is free once every MMA is done
+        else if (i < so.len) st_global_row32(p.dq, p.sdq, so, i, h, c * 32, w);
       }
     }
     fence_proxy_async_smem();
     named_bar_sync(1, 128);
-    if (ok && r == 0) {
-      for (int c = 0; c < NCH; ++c) tma_store_4d(&p.tm_dq, smem_u32(sQ + c * 16384), c * 64, h, i0, b);
+    if (ok && tile_store && r == 0) {
+      for (int c = 0; c < NCH; ++c)
+        tma_store_4d(&p.tm_dq, smem_u32(sQ + c * 16384), c * 64, h, so.row0 + i0, so.bt);
       bulk_commit();
       bulk_wait_all();
     }

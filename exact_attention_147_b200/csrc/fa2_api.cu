@@ -13,6 +13,8 @@
 #include <cstring>
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
+#include <utility>
 
 #include "../../include/fa2.h"
 #include "attn_common.cuh"
@@ -169,6 +171,22 @@ fa2_status encode_dqacc_3d(CUtensorMap* m, void* ptr, int B, int N, int H, int d
 
 Strides to_s(const fa2_strides& s) { return Strides{s.b, s.n, s.h}; }
 
+// The tensors as the TMA maps see them: B x N rows (padded) or one batch
+// entry of `total` rows (packed, whose b stride is unused and is given a
+// value that keeps the map well formed).
+struct MapShape {
+  int bt, rows;
+};
+MapShape map_shape(const AttnArgs& a) { return a.cu_seqlens ? MapShape{1, a.total} : MapShape{a.B, a.N}; }
+fa2_strides map_strides(const AttnArgs& a, fa2_strides s) {
+  if (a.cu_seqlens) s.b = s.n * int64_t(a.total > 0 ? a.total : 1);
+  return s;
+}
+fa2_status encode_input(CUtensorMap* m, const void* ptr, const fa2_strides& s, const AttnArgs& a, int d) {
+  const MapShape ms = map_shape(a);
+  return encode_bf16_4d(m, ptr, map_strides(a, s), ms.bt, ms.rows, a.H, d, 128);
+}
+
 void normalise_window(int causal, int* wl, int* wr) {
   if (*wl < 0) *wl = -1;
   if (*wr < 0) *wr = -1;
@@ -185,27 +203,53 @@ fa2_status launched(int n) {
   return FA2_OK;
 }
 
+// Work counters of the packed forward's dynamic scheduler: pairs of
+// {next unit, finished CTAs}, zero between calls (each call's last CTA resets
+// its pair).  Calls take the pairs round robin, so up to kSchedSlots packed
+// forward calls may run at the same time on different streams.
+constexpr int kSchedSlots = 64;
+static __device__ unsigned int g_fa2_sched[2 * kSchedSlots];
+unsigned int* g_sched_addr[kMaxDevices] = {};
+std::mutex g_sched_mu;
+std::atomic<uint32_t> g_sched_ticket{0};
+
+fa2_status sched_counters(int dev, unsigned int** out) {
+  {
+    std::lock_guard<std::mutex> lk(g_sched_mu);
+    if (g_sched_addr[dev] == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_fa2_sched) != cudaSuccess || ptr == nullptr) return FA2_ERR_CUDA;
+      g_sched_addr[dev] = static_cast<unsigned int*>(ptr);
+    }
+  }
+  *out = g_sched_addr[dev] + 2 * (g_sched_ticket.fetch_add(1) % kSchedSlots);
+  return FA2_OK;
+}
+
 template <int HD>
 fa2_status dispatch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
                               const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
                               int causal_order, cudaStream_t st);
 
-template <int HD, bool ALIBI, bool DROPOUT>
+template <int HD, bool ALIBI, bool DROPOUT, bool PACKED>
 fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
                             const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
                             int causal_order, cudaStream_t st) {
   static std::atomic<uint64_t> mask{0};
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
-  FA2_TRY(encode_bf16_4d(&p.tm_q, a.q, sq, a.B, a.N, a.H, HD, 128));
-  FA2_TRY(encode_bf16_4d(&p.tm_k, a.k, sk, a.B, a.N, a.H, HD, 128));
-  FA2_TRY(encode_bf16_4d(&p.tm_v, a.v, sv, a.B, a.N, a.H, HD, 128));
+  FA2_TRY(encode_input(&p.tm_q, a.q, sq, a, HD));
+  FA2_TRY(encode_input(&p.tm_k, a.k, sk, a, HD));
+  FA2_TRY(encode_input(&p.tm_v, a.v, sv, a, HD));
   p.o = static_cast<__nv_bfloat16*>(a.o);
-  p.so_b = so.b;
+  p.so_b = a.cu_seqlens ? 0 : so.b;
   p.so_n = so.n;
   p.so_h = so.h;
   p.lse = a.lse;
   p.alibi = a.alibi;
+  p.cu_seqlens = a.cu_seqlens;
+  p.total = a.total;
+  p.stat_rows = map_shape(a).rows;
   p.N = a.N;
   p.H = a.H;
   p.B = a.B;
@@ -217,7 +261,8 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.wait_ns = g_wait_ns.load();
   p.drop = a.drop;
-  auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT>;
+  if (PACKED) FA2_TRY(sched_counters(dev, &p.sched));
+  auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, PACKED>;
   constexpr int smem = FwdCfg<HD>::SMEM_BYTES;
   FA2_TRY(ensure_smem(kern, smem, dev, mask));
   // persistent grid: one CTA per SM (shared memory and TMEM allow one)
@@ -226,7 +271,7 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   return launched(1);
 }
 
-template <int HD, bool ALIBI, bool DROPOUT>
+template <int HD, bool ALIBI, bool DROPOUT, bool PACKED>
 fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
                             const fa2_strides& sv, const fa2_strides& sdo, const fa2_strides& sdq,
                             const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
@@ -234,24 +279,36 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   static std::atomic<uint64_t> mask_dkdv{0}, mask_dkdv_nodq{0}, mask_dq{0};
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
-  FA2_TRY(encode_bf16_4d(&p.tm_q, a.q, sq, a.B, a.N, a.H, HD, 128));
-  FA2_TRY(encode_bf16_4d(&p.tm_k, a.k, sk, a.B, a.N, a.H, HD, 128));
-  FA2_TRY(encode_bf16_4d(&p.tm_v, a.v, sv, a.B, a.N, a.H, HD, 128));
-  FA2_TRY(encode_bf16_4d(&p.tm_do, a.dout, sdo, a.B, a.N, a.H, HD, 128));
-  FA2_TRY(encode_bf16_4d(&p.tm_dq, a.dq, sdq, a.B, a.N, a.H, HD, 128));
-  FA2_TRY(encode_bf16_4d(&p.tm_dk, a.dk, sdk, a.B, a.N, a.H, HD, 128));
-  FA2_TRY(encode_bf16_4d(&p.tm_dv, a.dv, sdv, a.B, a.N, a.H, HD, 128));
-  if (!deterministic) FA2_TRY(encode_dqacc_3d(&p.tm_dqacc, a.dq_accum, a.B, a.N, a.H, HD));
+  const MapShape ms = map_shape(a);
+  FA2_TRY(encode_input(&p.tm_q, a.q, sq, a, HD));
+  FA2_TRY(encode_input(&p.tm_k, a.k, sk, a, HD));
+  FA2_TRY(encode_input(&p.tm_v, a.v, sv, a, HD));
+  FA2_TRY(encode_input(&p.tm_do, a.dout, sdo, a, HD));
+  FA2_TRY(encode_input(&p.tm_dq, a.dq, sdq, a, HD));
+  FA2_TRY(encode_input(&p.tm_dk, a.dk, sdk, a, HD));
+  FA2_TRY(encode_input(&p.tm_dv, a.dv, sdv, a, HD));
+  if (!deterministic) FA2_TRY(encode_dqacc_3d(&p.tm_dqacc, a.dq_accum, ms.bt, ms.rows, a.H, HD));
+  p.dq = static_cast<__nv_bfloat16*>(a.dq);
+  p.dk = static_cast<__nv_bfloat16*>(a.dk);
+  p.dv = static_cast<__nv_bfloat16*>(a.dv);
+  p.sdq = a.sdq;
+  p.sdk = a.sdk;
+  p.sdv = a.sdv;
   p.lse = a.lse;
   p.dvec = a.dvec;
   p.dq_accum = a.dq_accum;
   p.alibi = a.alibi;
+  p.cu_seqlens = a.cu_seqlens;
+  p.total = a.total;
+  p.stat_rows = ms.rows;
   p.N = a.N;
   p.H = a.H;
   p.B = a.B;
   p.wl = a.wl;
   p.wr = a.wr;
   p.nblocks = (a.N + 127) / 128;
+  // key blocks of one head next to each other (they share its Q and dO in
+  // L2) unless masks make the blocks' work vary
   p.heavy_first = (a.wr >= 0 || a.wl >= 0) ? 1 : 0;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
@@ -265,46 +322,62 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   // forever.  Refuse to launch otherwise.
   {
     cudaFuncAttributes fa;
-    auto k1c = deterministic ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT>
-                             : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT>;
+    auto k1c = deterministic ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, PACKED>
+                             : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, PACKED>;
     if (cudaFuncGetAttributes(&fa, k1c) != cudaSuccess) return FA2_ERR_CUDA;
     if (fa.numRegs < BwdCfg<HD>::REGS_AT_LAUNCH) return FA2_ERR_UNSUPPORTED;
   }
   if (!deterministic) {
-    const long long n4 = (long long)a.B * a.H * a.N * HD / 4;
+    const long long n4 = (long long)ms.bt * a.H * ms.rows * HD / 4;
     const unsigned zgrid = unsigned(std::min<long long>((n4 + 255) / 256, 148 * 16));
     zero_f32x4_kernel<<<zgrid, 256, 0, st>>>(reinterpret_cast<float4*>(a.dq_accum), n4);
     FA2_TRY(launched(1));
-    auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT>;
+    auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, PACKED>;
     FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv));
     k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
     FA2_TRY(launched(1));
-    const long long rows = (long long)a.B * a.H * a.N;
+    AttnArgs c = a;  // the accumulator is [bt * H, rows, d] in both layouts
+    c.B = ms.bt;
+    c.N = ms.rows;
+    c.cu_seqlens = nullptr;
+    const long long rows = (long long)c.B * c.H * c.N;
     const long long per_block = 256 / (HD / 4);
-    dq_convert_kernel<HD><<<unsigned((rows + per_block - 1) / per_block), 256, 0, st>>>(a);
+    dq_convert_kernel<HD><<<unsigned((rows + per_block - 1) / per_block), 256, 0, st>>>(c);
     return launched(1);
   }
-  auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT>;
+  auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, PACKED>;
   FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv_nodq));
   k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
   FA2_TRY(launched(1));
-  auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI, DROPOUT>;
+  auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI, DROPOUT, PACKED>;
   constexpr int smem2 = DqCfg<HD>::SMEM_BYTES;
   FA2_TRY(ensure_smem(k2, smem2, dev, mask_dq));
   k2<<<grid, DqCfg<HD>::THREADS, smem2, st>>>(p);
   return launched(1);
 }
 
+// Calls f(std::bool_constant<x>...) for the run-time flags x: picks the
+// kernel instantiation that matches the call's options.
+template <bool... Fixed, typename F>
+fa2_status static_bools(F&& f) {
+  return f(std::bool_constant<Fixed>{}...);
+}
+template <bool... Fixed, typename F, typename... Rest>
+fa2_status static_bools(F&& f, bool first, Rest... rest) {
+  return first ? static_bools<Fixed..., true>(f, rest...) : static_bools<Fixed..., false>(f, rest...);
+}
+
 template <int HD>
 fa2_status dispatch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
                               const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
                               int causal_order, cudaStream_t st) {
-  if (a.alibi) {
-    return a.dropout ? launch_fwd_sm100<HD, true, true>(a, sq, sk, sv, so, dev, sm_count, causal_order, st)
-                     : launch_fwd_sm100<HD, true, false>(a, sq, sk, sv, so, dev, sm_count, causal_order, st);
-  }
-  return a.dropout ? launch_fwd_sm100<HD, false, true>(a, sq, sk, sv, so, dev, sm_count, causal_order, st)
-                   : launch_fwd_sm100<HD, false, false>(a, sq, sk, sv, so, dev, sm_count, causal_order, st);
+  return static_bools(
+      [&](auto alibi, auto dropout, auto packed) {
+        return launch_fwd_sm100<HD, decltype(alibi)::value, decltype(dropout)::value,
+                                decltype(packed)::value>(a, sq, sk, sv, so, dev, sm_count,
+                                                         causal_order, st);
+      },
+      a.alibi != nullptr, a.dropout != 0, a.cu_seqlens != nullptr);
 }
 
 template <int HD>
@@ -312,12 +385,124 @@ fa2_status dispatch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa
                               const fa2_strides& sv, const fa2_strides& sdo, const fa2_strides& sdq,
                               const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
                               int dev, cudaStream_t st) {
-  if (a.alibi) {
-    return a.dropout ? launch_bwd_sm100<HD, true, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
-                     : launch_bwd_sm100<HD, true, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
+  return static_bools(
+      [&](auto alibi, auto dropout, auto packed) {
+        return launch_bwd_sm100<HD, decltype(alibi)::value, decltype(dropout)::value,
+                                decltype(packed)::value>(a, sq, sk, sv, sdo, sdq, sdk, sdv,
+                                                         deterministic, dev, st);
+      },
+      a.alibi != nullptr, a.dropout != 0, a.cu_seqlens != nullptr);
+}
+
+// ----------------------------------------------------------------- packed checks
+fa2_status check_packed_shape(const int32_t* cu, int B, int max_seqlen, int total, int H, int d,
+                              fa2_dtype dtype) {
+  if (cu == nullptr || (reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return FA2_ERR_INVALID_ARG;
+  if (max_seqlen < 1 || total < 0) return FA2_ERR_INVALID_ARG;
+  return check_shape(B, max_seqlen, H, d, dtype);
+}
+
+// A packed tensor [total, H, d]: only the row and head strides are used.
+fa2_status check_packed_tensor(const void* p, fa2_strides s, fa2_dtype dtype, int total) {
+  const int64_t lim = (int64_t(1) << 40) / (dtype == FA2_BF16 ? 2 : 4);
+  if (s.n >= 1 && int64_t(total) * s.n >= lim) return FA2_ERR_INVALID_ARG;
+  s.b = s.n;  // checked like the others, then ignored
+  return check_tensor(p, s, dtype);
+}
+
+fa2_status check_workspace(const void* ws, size_t bytes, size_t need) {
+  if (need == 0) return FA2_OK;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < need)
+    return FA2_ERR_INVALID_ARG;
+  return FA2_OK;
+}
+
+// ----------------------------------------------------------------- argument blocks
+void fill_common(AttnArgs* a, int B, int N, int H, int d, float softmax_scale, int causal,
+                 int window_left, int window_right, const float* alibi, float dropout_p,
+                 unsigned long long dropout_seed) {
+  a->B = B; a->N = N; a->H = H; a->d = d;
+  a->alibi = alibi;
+  a->scale = resolve_scale(softmax_scale, d);
+  a->wl = window_left;
+  a->wr = window_right;
+  normalise_window(causal, &a->wl, &a->wr);
+  a->dropout = dropout_p != 0.f;
+  a->drop = make_dropout(dropout_p, dropout_seed);
+}
+
+void fill_fwd_args(AttnArgs* a, const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int N, int H, int d, const fa2_strides& sq, const fa2_strides& sk,
+                   const fa2_strides& sv, const fa2_strides& so, float softmax_scale, int causal,
+                   int window_left, int window_right, const float* alibi, float dropout_p,
+                   unsigned long long dropout_seed) {
+  std::memset(a, 0, sizeof(*a));
+  a->q = q; a->k = k; a->v = v; a->o = o; a->lse = lse;
+  a->sq = to_s(sq); a->sk = to_s(sk); a->sv = to_s(sv); a->so = to_s(so);
+  fill_common(a, B, N, H, d, softmax_scale, causal, window_left, window_right, alibi, dropout_p,
+              dropout_seed);
+}
+
+void fill_bwd_args(AttnArgs* a, const void* q, const void* k, const void* v, const void* dout,
+                   const float* lse, const float* D, void* dq, void* dk, void* dv, void* workspace,
+                   int B, int N, int H, int d, const fa2_strides& sq, const fa2_strides& sk,
+                   const fa2_strides& sv, const fa2_strides& sdo, const fa2_strides& sdq,
+                   const fa2_strides& sdk, const fa2_strides& sdv, float softmax_scale, int causal,
+                   int window_left, int window_right, const float* alibi, float dropout_p,
+                   unsigned long long dropout_seed) {
+  std::memset(a, 0, sizeof(*a));
+  a->q = q; a->k = k; a->v = v; a->dout = dout;
+  a->lse = const_cast<float*>(lse); a->dvec = D;
+  a->dq = dq; a->dk = dk; a->dv = dv;
+  a->dq_accum = static_cast<float*>(workspace);
+  a->sq = to_s(sq); a->sk = to_s(sk); a->sv = to_s(sv); a->sdo = to_s(sdo);
+  a->sdq = to_s(sdq); a->sdk = to_s(sdk); a->sdv = to_s(sdv);
+  fill_common(a, B, N, H, d, softmax_scale, causal, window_left, window_right, alibi, dropout_p,
+              dropout_seed);
+}
+
+// ----------------------------------------------------------------- kernel choice
+fa2_status run_fwd(const AttnArgs& a, fa2_dtype dtype, const fa2_strides& sq, const fa2_strides& sk,
+                   const fa2_strides& sv, const fa2_strides& so, cudaStream_t st) {
+  int dev;
+  DeviceInfo di;
+  FA2_TRY(current_device(&dev, &di));
+  if (dtype == FA2_F32) {
+    dim3 grid((a.N + 3) / 4, a.H, a.B);
+    if (a.d == 64) simt_fwd_kernel<float, 64><<<grid, 128, 0, st>>>(a);
+    else simt_fwd_kernel<float, 128><<<grid, 128, 0, st>>>(a);
+    return launched(1);
   }
-  return a.dropout ? launch_bwd_sm100<HD, false, true>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
-                   : launch_bwd_sm100<HD, false, false>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
+  if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;  // sm_100a kernels only
+  // Longest-first unit order when masks make the work per unit vary;
+  // otherwise the query pairs of one head run together and share its K/V
+  // in L2.  (Packed calls take units dynamically in this order.)
+  const int heavy_first = (a.wr >= 0 || a.wl >= 0) ? 1 : 0;
+  return a.d == 128 ? dispatch_fwd_sm100<128>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st)
+                    : dispatch_fwd_sm100<64>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st);
+}
+
+fa2_status run_bwd(const AttnArgs& a, fa2_dtype dtype, const fa2_strides& sq, const fa2_strides& sk,
+                   const fa2_strides& sv, const fa2_strides& sdo, const fa2_strides& sdq,
+                   const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
+                   cudaStream_t st) {
+  int dev;
+  DeviceInfo di;
+  FA2_TRY(current_device(&dev, &di));
+  if (dtype == FA2_F32) {
+    dim3 grid((a.N + 3) / 4, a.H, a.B);
+    if (a.d == 64) {
+      simt_bwd_dkdv_kernel<float, 64><<<grid, 128, 0, st>>>(a);
+      simt_bwd_dq_kernel<float, 64><<<grid, 128, 0, st>>>(a);
+    } else {
+      simt_bwd_dkdv_kernel<float, 128><<<grid, 128, 0, st>>>(a);
+      simt_bwd_dq_kernel<float, 128><<<grid, 128, 0, st>>>(a);
+    }
+    return launched(2);
+  }
+  if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;
+  return a.d == 128 ? dispatch_bwd_sm100<128>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
+                    : dispatch_bwd_sm100<64>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
 }
 
 }  // namespace
@@ -330,7 +515,8 @@ const char* fa2_strerror(fa2_status s) {
     case FA2_ERR_INVALID_ARG: return "FA2_ERR_INVALID_ARG: invalid pointer, shape, stride or option";
     case FA2_ERR_UNSUPPORTED: return "FA2_ERR_UNSUPPORTED: valid but not implemented";
     case FA2_ERR_CUDA: return "FA2_ERR_CUDA: a CUDA call failed";
-    case FA2_ERR_DEVICE_TIMEOUT: return "FA2_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait";
+    case FA2_ERR_DEVICE_TIMEOUT:
+      return "FA2_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait or met malformed cu_seqlens";
     case FA2_ERR_SCRATCH_LIMIT:
       return "FA2_ERR_SCRATCH_LIMIT: B*H*N*d exceeds the fixed scratch of fa2_bwd_noalloc";
   }
@@ -371,34 +557,33 @@ fa2_status fa2_fwd(const void* q, const void* k, const void* v, void* o, float* 
   if (lse == nullptr || !aligned16(lse)) return FA2_ERR_INVALID_ARG;
   if (o == q || o == k || o == v) return FA2_ERR_INVALID_ARG;
   FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
-
   AttnArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.alibi = alibi_slopes;
-  a.sq = to_s(sq); a.sk = to_s(sk); a.sv = to_s(sv); a.so = to_s(so);
-  a.B = B; a.N = N; a.H = H; a.d = d;
-  a.scale = resolve_scale(softmax_scale, d);
-  a.wl = window_left;
-  a.wr = window_right;
-  normalise_window(causal, &a.wl, &a.wr);
-  a.dropout = dropout_p != 0.f;
-  a.drop = make_dropout(dropout_p, dropout_seed);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  fill_fwd_args(&a, q, k, v, o, lse, B, N, H, d, sq, sk, sv, so, softmax_scale, causal, window_left,
+                window_right, alibi_slopes, dropout_p, dropout_seed);
+  return run_fwd(a, dtype, sq, sk, sv, so, static_cast<cudaStream_t>(stream));
+}
 
-  int dev;
-  DeviceInfo di;
-  FA2_TRY(current_device(&dev, &di));
-
-  if (dtype == FA2_F32) {
-    dim3 grid((N + 3) / 4, H, B);
-    if (d == 64) simt_fwd_kernel<float, 64><<<grid, 128, 0, st>>>(a);
-    else simt_fwd_kernel<float, 128><<<grid, 128, 0, st>>>(a);
-    return launched(1);
-  }
-  if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;  // sm_100a kernels only
-  const int heavy_first = (a.wr >= 0 || a.wl >= 0) ? 1 : 0;
-  return d == 128 ? dispatch_fwd_sm100<128>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st)
-                  : dispatch_fwd_sm100<64>(a, sq, sk, sv, so, dev, di.sm_count, heavy_first, st);
+fa2_status fa2_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const int32_t* cu_seqlens, int B, int max_seqlen, int total, int H, int d,
+                          fa2_dtype dtype, fa2_strides sq, fa2_strides sk, fa2_strides sv,
+                          fa2_strides so, float softmax_scale, int causal, int window_left,
+                          int window_right, const float* alibi_slopes, float dropout_p,
+                          unsigned long long dropout_seed, void* stream) {
+  FA2_TRY(check_packed_shape(cu_seqlens, B, max_seqlen, total, H, d, dtype));
+  FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
+  if (total == 0) return FA2_OK;  // every sequence is empty
+  FA2_TRY(check_packed_tensor(q, sq, dtype, total));
+  FA2_TRY(check_packed_tensor(k, sk, dtype, total));
+  FA2_TRY(check_packed_tensor(v, sv, dtype, total));
+  FA2_TRY(check_packed_tensor(o, so, dtype, total));
+  if (lse == nullptr || !aligned16(lse)) return FA2_ERR_INVALID_ARG;
+  if (o == q || o == k || o == v) return FA2_ERR_INVALID_ARG;
+  AttnArgs a;
+  fill_fwd_args(&a, q, k, v, o, lse, B, max_seqlen, H, d, sq, sk, sv, so, softmax_scale, causal,
+                window_left, window_right, alibi_slopes, dropout_p, dropout_seed);
+  a.cu_seqlens = cu_seqlens;
+  a.total = total;
+  return run_fwd(a, dtype, sq, sk, sv, so, static_cast<cudaStream_t>(stream));
 }
 
 fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D, int B, int N, int H, int d,
@@ -446,53 +631,47 @@ fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout
                    float dropout_p, unsigned long long dropout_seed, int deterministic,
                    void* stream) {
   FA2_TRY(check_shape(B, N, H, d, dtype));
-  FA2_TRY(check_tensor(q, sq, dtype));
-  FA2_TRY(check_tensor(k, sk, dtype));
-  FA2_TRY(check_tensor(v, sv, dtype));
-  FA2_TRY(check_tensor(dout, sdo, dtype));
-  FA2_TRY(check_tensor(dq, sdq, dtype));
-  FA2_TRY(check_tensor(dk, sdk, dtype));
-  FA2_TRY(check_tensor(dv, sdv, dtype));
+  for (auto [ptr, s] : {std::pair<const void*, fa2_strides>{q, sq}, {k, sk}, {v, sv}, {dout, sdo},
+                        {dq, sdq}, {dk, sdk}, {dv, sdv}})
+    FA2_TRY(check_tensor(ptr, s, dtype));
   if (lse == nullptr || !aligned16(lse) || D == nullptr || !aligned16(D)) return FA2_ERR_INVALID_ARG;
   FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
-  const size_t need = fa2_bwd_workspace_size(B, N, H, d, dtype, deterministic);
-  if (need > 0) {
-    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-        workspace_bytes < need)
-      return FA2_ERR_INVALID_ARG;
-  }
+  FA2_TRY(check_workspace(workspace, workspace_bytes,
+                          fa2_bwd_workspace_size(B, N, H, d, dtype, deterministic)));
   AttnArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = const_cast<float*>(lse); a.dvec = D;
-  a.dq = dq; a.dk = dk; a.dv = dv; a.alibi = alibi_slopes;
-  a.dq_accum = static_cast<float*>(workspace);
-  a.sq = to_s(sq); a.sk = to_s(sk); a.sv = to_s(sv); a.sdo = to_s(sdo);
-  a.sdq = to_s(sdq); a.sdk = to_s(sdk); a.sdv = to_s(sdv);
-  a.B = B; a.N = N; a.H = H; a.d = d;
-  a.scale = resolve_scale(softmax_scale, d);
-  a.wl = window_left;
-  a.wr = window_right;
-  normalise_window(causal, &a.wl, &a.wr);
-  a.dropout = dropout_p != 0.f;
-  a.drop = make_dropout(dropout_p, dropout_seed);
-  int dev;
-  DeviceInfo di;
-  FA2_TRY(current_device(&dev, &di));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  dim3 grid((N + 3) / 4, H, B);
-  if (dtype == FA2_F32) {
-    if (d == 64) {
-      simt_bwd_dkdv_kernel<float, 64><<<grid, 128, 0, st>>>(a);
-      simt_bwd_dq_kernel<float, 64><<<grid, 128, 0, st>>>(a);
-    } else {
-      simt_bwd_dkdv_kernel<float, 128><<<grid, 128, 0, st>>>(a);
-      simt_bwd_dq_kernel<float, 128><<<grid, 128, 0, st>>>(a);
-    }
-    return launched(2);
-  }
-  if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;
-  return d == 128 ? dispatch_bwd_sm100<128>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st)
-                  : dispatch_bwd_sm100<64>(a, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic, dev, st);
+  fill_bwd_args(&a, q, k, v, dout, lse, D, dq, dk, dv, workspace, B, N, H, d, sq, sk, sv, sdo, sdq,
+                sdk, sdv, softmax_scale, causal, window_left, window_right, alibi_slopes, dropout_p,
+                dropout_seed);
+  return run_bwd(a, dtype, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic,
+                 static_cast<cudaStream_t>(stream));
+}
+
+fa2_status fa2_bwd_varlen(const void* q, const void* k, const void* v, const void* dout,
+                          const float* lse, const float* D, void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes, const int32_t* cu_seqlens, int B,
+                          int max_seqlen, int total, int H, int d, fa2_dtype dtype, fa2_strides sq,
+                          fa2_strides sk, fa2_strides sv, fa2_strides sdo, fa2_strides sdq,
+                          fa2_strides sdk, fa2_strides sdv, float softmax_scale, int causal,
+                          int window_left, int window_right, const float* alibi_slopes,
+                          float dropout_p, unsigned long long dropout_seed, int deterministic,
+                          void* stream) {
+  FA2_TRY(check_packed_shape(cu_seqlens, B, max_seqlen, total, H, d, dtype));
+  FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
+  if (total == 0) return FA2_OK;
+  for (auto [ptr, s] : {std::pair<const void*, fa2_strides>{q, sq}, {k, sk}, {v, sv}, {dout, sdo},
+                        {dq, sdq}, {dk, sdk}, {dv, sdv}})
+    FA2_TRY(check_packed_tensor(ptr, s, dtype, total));
+  if (lse == nullptr || !aligned16(lse) || D == nullptr || !aligned16(D)) return FA2_ERR_INVALID_ARG;
+  FA2_TRY(check_workspace(workspace, workspace_bytes,
+                          fa2_bwd_workspace_size(1, total, H, d, dtype, deterministic)));
+  AttnArgs a;
+  fill_bwd_args(&a, q, k, v, dout, lse, D, dq, dk, dv, workspace, B, max_seqlen, H, d, sq, sk, sv,
+                sdo, sdq, sdk, sdv, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                dropout_p, dropout_seed);
+  a.cu_seqlens = cu_seqlens;
+  a.total = total;
+  return run_bwd(a, dtype, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic,
+                 static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -550,21 +729,10 @@ fa2_status fa2_bwd_noalloc(const void* q, const void* k, const void* v, const vo
   if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;
   float* scratch = nullptr;
   FA2_TRY(noalloc_scratch(dev, &scratch));
-  AttnArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.q = q; a.k = k; a.v = v; a.dout = dout; a.lse = const_cast<float*>(lse); a.dvec = D;
-  a.dq = dq; a.dk = dk; a.dv = dv; a.alibi = alibi_slopes;
-  a.dq_accum = scratch;  // cleared by the first kernel of the launch sequence
-  a.sq = to_s(sq); a.sk = to_s(sk); a.sv = to_s(sv); a.sdo = to_s(sdo);
-  a.sdq = to_s(sdq); a.sdk = to_s(sdk); a.sdv = to_s(sdv);
-  a.B = B; a.N = N; a.H = H; a.d = d;
-  a.scale = resolve_scale(softmax_scale, d);
-  a.wl = window_left;
-  a.wr = window_right;
-  normalise_window(causal, &a.wl, &a.wr);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 128 ? dispatch_bwd_sm100<128>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st)
-                  : dispatch_bwd_sm100<64>(a, sq, sk, sv, sdo, sdq, sdk, sdv, 0, dev, st);
+  AttnArgs a;  // the scratch is cleared by the first kernel of the launch sequence
+  fill_bwd_args(&a, q, k, v, dout, lse, D, dq, dk, dv, scratch, B, N, H, d, sq, sk, sv, sdo, sdq,
+                sdk, sdv, softmax_scale, causal, window_left, window_right, alibi_slopes, 0.f, 0);
+  return run_bwd(a, dtype, sq, sk, sv, sdo, sdq, sdk, sdv, 0, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -45,6 +45,12 @@
 // range (fully hidden blocks are never loaded); inside a block, a row that is
 // not entirely visible masks element-wise.  The tail beyond N is zero-filled
 // by TMA and masked the same way.
+//
+// Packed (variable-length) batches: a unit addresses its sequence's rows
+// through the tensor-row offset of that sequence.  Tiles that run past the
+// end of the sequence read the next sequence's rows; those keys are masked
+// like any invisible key and those query rows are never stored, so the
+// result is the one each sequence would get alone.
 #pragma once
 
 #include <math_constants.h>
@@ -57,11 +63,15 @@ namespace fa2 {
 
 struct FwdParams {
   CUtensorMap tm_q, tm_k, tm_v;        // [B,N,H,d] bf16, box {64,1,128,1}, 128B swizzle
-  __nv_bfloat16* o;                    // [B,N,H,d] output
+                                       // (packed: [1,total,H,d])
+  __nv_bfloat16* o;                    // [B,N,H,d] / [total,H,d] output
   long long so_b, so_n, so_h;          // its element strides
-  float* lse;                          // [B,H,N]
+  float* lse;                          // [B,H,N] / [H,total]
   const float* alibi;                  // [H] or null
-  int N, H, B;
+  const int* cu_seqlens;               // [B+1] sequence offsets (packed) or null (padded)
+  int total;                           // packed: tensor rows
+  int stat_rows;                       // rows per (batch, head) of lse: N or total
+  int N, H, B;                         // N: the (longest) sequence length
   int wl, wr;                          // inclusive window, negative = unbounded
   int npairs;                          // ceil(N / 256)
   int num_units;                       // npairs * H * B
@@ -69,6 +79,7 @@ struct FwdParams {
   float scale_log2;                    // softmax_scale * log2(e)
   unsigned long long wait_ns;          // bounded-wait limit
   DropoutParams drop;                  // used by the DROPOUT instantiations
+  unsigned int* sched;                 // packed: {next unit, finished CTAs}, 0 between calls
 };
 
 template <int HD>
@@ -82,10 +93,12 @@ struct FwdCfg {
   static constexpr int KV_BYTES = BN * HD * 2;
   static constexpr int OFF_KV = QBUFS * NQT * QT_BYTES;
   static constexpr int OFF_BARS = OFF_KV + SLOTS * KV_BYTES;
+  static constexpr int RING = 4;        // unit-index ring of the packed scheduler
   // q_full[2], q_empty[2], slot full/empty, s_full[2], p_ready[2], o_full[2],
-  // o_empty[2], drain
-  static constexpr int NBARS = 2 * QBUFS + 2 * SLOTS + 4 * NQT + 1;
-  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16;
+  // o_empty[2], drain, ring full[4], ring empty[4]
+  static constexpr int NBARS = 2 * QBUFS + 2 * SLOTS + 4 * NQT + 1 + 2 * RING;
+  // barriers, then the TMEM address, the abort flag, 2 spare words and the ring
+  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16 + 4 * RING;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static constexpr int THREADS = 320;
 };
@@ -98,36 +111,70 @@ constexpr float LOG2E = 1.44269504088896340736f;
 constexpr int SITE_PROD = 0x100, SITE_MMA = 0x200, SITE_SOFT = 0x300, SITE_DRAIN = 0x400;
 constexpr int SITE_SMEM_ALIGN_F = 0xF01;
 
-// The k-th unit of CTA c in a persistent grid of G CTAs: round k covers
-// units [kG, kG + G) of the longest-first order, walked forwards in even
-// rounds and backwards in odd rounds, so each CTA's heavy and light units
-// pair up when the work per unit varies (causal and sliding-window masks).
+// Padded calls: the k-th unit of CTA c in a persistent grid of G CTAs.
+// Round k covers units [kG, kG + G) of the longest-first order, walked
+// forwards in even rounds and backwards in odd rounds, so each CTA's heavy
+// and light units pair up when the work per unit varies (causal and
+// sliding-window masks).  With equal sequence lengths this static schedule
+// is within a few percent of the best one.
 __device__ __forceinline__ int unit_index(int k) {
   const int G = int(gridDim.x), c = int(blockIdx.x);
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-// Unit index -> (query pair, batch*H + head, first KV block, KV block count).
+// Unit index -> (head, sequence, its rows, first local query row, first KV
+// block, KV block count).  A unit whose query pair lies past the end of its
+// sequence (packed calls: shorter sequences) has nblk = 0.
 struct Unit {
-  int pair, hb, row0, blk_begin, nblk;
+  int h, b, bt, base, len, row0, blk_begin, nblk;
 };
+template <bool PACKED>
 __device__ __forceinline__ Unit unit_of(const FwdParams& p, int L) {
   Unit u;
   const int nhb = p.H * p.B;
+  int pair, hb;
   if (p.heavy_first) {
-    u.pair = p.npairs - 1 - L / nhb;
-    u.hb = L % nhb;
+    pair = p.npairs - 1 - L / nhb;
+    hb = L % nhb;
   } else {
-    u.pair = L % p.npairs;
-    u.hb = L / p.npairs;
+    pair = L % p.npairs;
+    hb = L / p.npairs;
   }
-  u.row0 = u.pair * 256;
-  const int row_end = min(p.N, u.row0 + 256);
-  const int kv_lo = p.wl >= 0 ? max(0, u.row0 - p.wl) : 0;
-  const int kv_hi = p.wr >= 0 ? min(p.N - 1, row_end - 1 + p.wr) : p.N - 1;
-  u.blk_begin = kv_lo / 128;
-  u.nblk = kv_hi / 128 - u.blk_begin + 1;
+  u.h = hb % p.H;
+  u.b = hb / p.H;
+  if (PACKED) {
+    const SeqView sv = seq_view(p.cu_seqlens, u.b, p.N, p.total);
+    u.bt = sv.bt;
+    u.base = sv.row0;
+    u.len = sv.len;
+  } else {
+    u.bt = u.b;
+    u.base = 0;
+    u.len = p.N;
+  }
+  u.row0 = pair * 256;
+  u.blk_begin = 0;
+  u.nblk = 0;
+  if (u.row0 < u.len) {
+    const int row_end = min(u.len, u.row0 + 256);
+    const int kv_lo = p.wl >= 0 ? max(0, u.row0 - p.wl) : 0;
+    const int kv_hi = p.wr >= 0 ? min(u.len - 1, row_end - 1 + p.wr) : u.len - 1;
+    u.blk_begin = kv_lo / 128;
+    u.nblk = kv_hi / 128 - u.blk_begin + 1;
+  }
   return u;
+}
+// Packed calls: units differ in cost with the sequence lengths, which a
+// static schedule cannot see, so the CTAs take units from a shared counter in
+// longest-first order, each as it becomes free.  Returns the next non-empty
+// unit, or -1 when none is left.  Only the producer thread calls this.
+template <bool PACKED>
+__device__ __forceinline__ int fetch_unit(const FwdParams& p) {
+  for (;;) {
+    const int L = int(atomicAdd(p.sched, 1u));
+    if (L >= p.num_units) return -1;
+    if (unit_of<PACKED>(p, L).nblk > 0) return L;
+  }
 }
 }  // namespace fwd_detail
 
@@ -143,7 +190,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-template <int HD, bool ALIBI, bool DROPOUT>
+template <int HD, bool ALIBI, bool DROPOUT, bool PACKED>
 __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<HD>;
   constexpr int BM = C::BM, BN = C::BN, NQT = C::NQT, SLOTS = C::SLOTS;
@@ -168,8 +215,11 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
   auto o_full = [&](int t) { return bar0 + 8u * (8 + 2 * SLOTS + t); };
   auto o_empty = [&](int t) { return bar0 + 8u * (10 + 2 * SLOTS + t); };
   const uint32_t drain_bar = bar0 + 8u * (12 + 2 * SLOTS);
+  auto ring_full = [&](int r) { return bar0 + 8u * (13 + 2 * SLOTS + r); };
+  auto ring_empty = [&](int r) { return bar0 + 8u * (13 + 2 * SLOTS + C::RING + r); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* ring = abort_flag + 3;  // packed: unit indices handed from the producer to the other roles
   AbortFlag ab{abort_flag};
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -178,9 +228,10 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
     *abort_flag = 0;
     for (int i = 0; i < C::NBARS; ++i) {
       const uint32_t bar = bar0 + 8u * i;
-      bar_init(bar, (bar == p_ready(0) || bar == p_ready(1) || bar == o_empty(0) || bar == o_empty(1))
-                        ? 128
-                        : 1);
+      uint32_t cnt = 1;
+      if (bar == p_ready(0) || bar == p_ready(1) || bar == o_empty(0) || bar == o_empty(1)) cnt = 128;
+      if (bar >= ring_empty(0) && bar <= ring_empty(C::RING - 1)) cnt = 9;  // MMA + 8 softmax warps
+      bar_init(bar, cnt);
     }
     fence_barrier_init();
   }
@@ -203,19 +254,29 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
     if (lane == 0) {
       int n = 0, k = 0, q_issued = 0;
       bool ok = true;
-      for (int L = unit_index(0); L < p.num_units && ok; L = unit_index(++k)) {
-        const Unit u = unit_of(p, L);
-        const int h = u.hb % p.H, b = u.hb / p.H;
+      int L = PACKED ? fetch_unit<PACKED>(p) : unit_index(0);
+      for (;; ++k) {
+        if (PACKED) {  // hand the unit index (or the end mark -1) to the other roles
+          const int r = k % C::RING;
+          if (!wait_bar(ring_empty(r), ((k / C::RING) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + 3)) break;
+          ring[r] = L;
+          bar_arrive(ring_full(r));
+          if (L < 0) break;
+        } else if (L >= p.num_units) {
+          break;
+        }
+        const Unit u = unit_of<PACKED>(p, L);
+        const int L_next = PACKED ? fetch_unit<PACKED>(p) : unit_index(k + 1);
         const int qb = k & 1;
         if (!wait_bar(q_empty(qb), ((k >> 1) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + 2)) break;
         bar_arrive_expect_tx(q_full(qb), NQT * C::QT_BYTES);
         for (int t = 0; t < NQT; ++t)
           for (int c = 0; c < NCH; ++c)
             tma_load_4d(smem_u32(sQ + (qb * NQT + t) * C::QT_BYTES + c * BM * 128), &p.tm_q, q_full(qb),
-                        c * 64, h, u.row0 + t * BM, b);
+                        c * 64, u.h, u.base + u.row0 + t * BM, u.bt);
         q_issued = k + 1;
         for (int it = 0; it < u.nblk && ok; ++it) {
-          const int kv0 = (u.blk_begin + it) * BN;
+          const int kv0 = u.base + (u.blk_begin + it) * BN;
           for (int which = 0; which < 2; ++which, ++n) {
             const int s = n % SLOTS;
             if (!wait_bar(slot_empty(s), ((n / SLOTS) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + which)) {
@@ -225,8 +286,21 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
             bar_arrive_expect_tx(slot_full(s), C::KV_BYTES);
             const CUtensorMap* tm = which == 0 ? &p.tm_k : &p.tm_v;
             for (int c = 0; c < NCH; ++c)
-              tma_load_4d(smem_u32(sKV + s * C::KV_BYTES + c * BN * 128), tm, slot_full(s), c * 64, h, kv0, b);
+              tma_load_4d(smem_u32(sKV + s * C::KV_BYTES + c * BN * 128), tm, slot_full(s), c * 64, u.h, kv0,
+                          u.bt);
           }
+        }
+        if (!ok) break;
+        L = L_next;
+      }
+      if (PACKED) {
+        // The last CTA to finish taking units returns the counters to zero
+        // for the next call that uses them.
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+          p.sched[0] = 0u;
+          p.sched[1] = 0u;
+          __threadfence();
         }
       }
       // Before the CTA may exit, every copy issued must have landed.
@@ -256,10 +330,22 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
           umma_ts(tmem + 256 + t * HD, tmem + t * 128 + kk * 8,
                   sdesc_sw128(v0 + kk * 2048, BN * 128, 1024), id_pv, (acc || kk > 0) ? 1u : 0u);
       };
-      int n = 0, k = 0, g = 0;  // KV slot counter, unit counter, block counter
+      int n = 0, g = 0;  // KV slots, blocks
       bool ok = true;
-      for (int L = unit_index(0); L < p.num_units && ok; L = unit_index(++k)) {
-        const Unit u = unit_of(p, L);
+      for (int k = 0; ok; ++k) {
+        int L;
+        if (PACKED) {
+          const int r = k % C::RING;
+          ok = wait_bar(ring_full(r), (k / C::RING) & 1, ab, p.wait_ns, SITE_MMA + 8);
+          if (!ok) break;
+          L = ring[r];
+          bar_arrive(ring_empty(r));
+          if (L < 0) break;
+        } else {
+          L = unit_index(k);
+          if (L >= p.num_units) break;
+        }
+        const Unit u = unit_of<PACKED>(p, L);
         const int qb = k & 1;
         ok = wait_bar(q_full(qb), (k >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
         if (!ok) break;
@@ -330,14 +416,27 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
     const uint32_t s_addr = tmem + lane_base + t * 128;
     const uint32_t o_addr = tmem + lane_base + 256 + t * HD;
     const float C2 = p.scale_log2;
-    int g = 0, k = 0;
+    int g = 0;
     bool ok = true;
-    for (int L = unit_index(0); L < p.num_units && ok; L = unit_index(++k)) {
-      const Unit u = unit_of(p, L);
-      const int h = u.hb % p.H, b = u.hb / p.H;
-      const int i = u.row0 + t * BM + r;  // query row (>= N for padding rows)
+    for (int k = 0; ok; ++k) {
+      int L;
+      if (PACKED) {
+        const int r = k % C::RING;
+        ok = wait_bar(ring_full(r), (k / C::RING) & 1, ab, p.wait_ns, SITE_SOFT + 2);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        L = ring[r];
+        __syncwarp();
+        if (lane == 0) bar_arrive(ring_empty(r));
+        if (L < 0) break;
+      } else {
+        L = unit_index(k);
+        if (L >= p.num_units) break;
+      }
+      const Unit u = unit_of<PACKED>(p, L);
+      const int h = u.h, b = u.b;
+      const int i = u.row0 + t * BM + r;  // local query row (>= len for padding rows)
       const int lo = p.wl >= 0 ? max(0, i - p.wl) : 0;
-      const int hi = p.wr >= 0 ? min(p.N - 1, i + p.wr) : p.N - 1;
+      const int hi = p.wr >= 0 ? min(u.len - 1, i + p.wr) : u.len - 1;
       float slope2 = 0.f;
       if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
       float m_run = -CUDART_INF_F, l_run = 0.f;
@@ -446,7 +545,10 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
       if (!ok) break;
       tc_fence_after();
       const float inv_l = l_run > 0.f ? (DROPOUT ? p.drop.keep_scale : 1.f) / l_run : 0.f;
-      __nv_bfloat16* orow = p.o + b * p.so_b + (long long)i * p.so_n + h * p.so_h;
+      // the sequence's rows, looked up again here rather than kept live
+      // through the block loop
+      const SeqView sv = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};
+      __nv_bfloat16* orow = p.o + sv.bt * p.so_b + (long long)(sv.row0 + i) * p.so_n + h * p.so_h;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t w32[32];
@@ -460,15 +562,15 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           w16[e] = pack_bf16(__uint_as_float(w32[2 * e]) * inv_l, __uint_as_float(w32[2 * e + 1]) * inv_l);
-        if (i < p.N) {
+        if (i < sv.len) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
             *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) =
                 make_uint4(w16[4 * q4], w16[4 * q4 + 1], w16[4 * q4 + 2], w16[4 * q4 + 3]);
         }
       }
-      if (i < p.N)
-        p.lse[(size_t(b) * p.H + h) * p.N + i] =
+      if (i < sv.len)
+        p.lse[(size_t(sv.bt) * p.H + h) * (PACKED ? p.stat_rows : p.N) + sv.row0 + i] =
             l_run > 0.f ? (m_run + log2f(l_run)) * LN2 : -CUDART_INF_F;
       g += u.nblk;
     }

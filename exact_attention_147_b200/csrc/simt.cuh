@@ -48,17 +48,18 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(const AttnArgs a) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int i = blockIdx.x * 4 + warp;
   const int h = blockIdx.y, b = blockIdx.z;
-  if (i >= a.N) return;
-  const T* q = static_cast<const T*>(a.q) + b * a.sq.b + i * a.sq.n + h * a.sq.h;
-  const T* kb = static_cast<const T*>(a.k) + b * a.sk.b + h * a.sk.h;
-  const T* vb = static_cast<const T*>(a.v) + b * a.sv.b + h * a.sv.h;
+  const SeqView sv = seq_view(a.cu_seqlens, b, a.N, a.total);
+  if (i >= sv.len) return;
+  const T* q = row_ptr<const T>(a.q, a.sq, sv, i, h);
+  const T* kb = row_ptr<const T>(a.k, a.sk, sv, 0, h);
+  const T* vb = row_ptr<const T>(a.v, a.sv, sv, 0, h);
   float qr[E], acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     qr[e] = to_f(q[lane + 32 * e]);
     acc[e] = 0.f;
   }
-  const int lo = visible_lo(a, i), hi = visible_hi(a, i);
+  const int lo = visible_lo(a, i), hi = visible_hi(a, i, sv.len);
   const float slope = a.alibi ? a.alibi[h] : 0.f;
   float m = -CUDART_INF_F, l = 0.f;
   for (int j = lo; j <= hi; ++j) {
@@ -82,11 +83,11 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(const AttnArgs a) {
     for (int e = 0; e < E; ++e) acc[e] = fmaf(pk, to_f(vr[lane + 32 * e]), acc[e] * alpha);
     m = m_new;
   }
-  T* o = static_cast<T*>(a.o) + b * a.so.b + i * a.so.n + h * a.so.h;
+  T* o = row_ptr<T>(a.o, a.so, sv, i, h);
   const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
   for (int e = 0; e < E; ++e) o[lane + 32 * e] = from_f<T>(acc[e] * inv);
-  if (lane == 0) a.lse[(size_t(b) * a.H + h) * a.N + i] = l > 0.f ? m + logf(l) : -CUDART_INF_F;
+  if (lane == 0) a.lse[stat_index(a, sv, h, i)] = l > 0.f ? m + logf(l) : -CUDART_INF_F;
 }
 
 // dK, dV: warp per key row j; loops over the queries that see key j.
@@ -96,13 +97,14 @@ __global__ void __launch_bounds__(128) simt_bwd_dkdv_kernel(const AttnArgs a) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int j = blockIdx.x * 4 + warp;
   const int h = blockIdx.y, b = blockIdx.z;
-  if (j >= a.N) return;
-  const T* kr = static_cast<const T*>(a.k) + b * a.sk.b + j * a.sk.n + h * a.sk.h;
-  const T* vr = static_cast<const T*>(a.v) + b * a.sv.b + j * a.sv.n + h * a.sv.h;
-  const T* qb = static_cast<const T*>(a.q) + b * a.sq.b + h * a.sq.h;
-  const T* dob = static_cast<const T*>(a.dout) + b * a.sdo.b + h * a.sdo.h;
-  const float* lse = a.lse + (size_t(b) * a.H + h) * a.N;
-  const float* dvec = a.dvec + (size_t(b) * a.H + h) * a.N;
+  const SeqView sv = seq_view(a.cu_seqlens, b, a.N, a.total);
+  if (j >= sv.len) return;
+  const T* kr = row_ptr<const T>(a.k, a.sk, sv, j, h);
+  const T* vr = row_ptr<const T>(a.v, a.sv, sv, j, h);
+  const T* qb = row_ptr<const T>(a.q, a.sq, sv, 0, h);
+  const T* dob = row_ptr<const T>(a.dout, a.sdo, sv, 0, h);
+  const float* lse = a.lse + stat_index(a, sv, h, 0);
+  const float* dvec = a.dvec + stat_index(a, sv, h, 0);
   float kf[E], vf[E], dk[E], dv[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(128) simt_bwd_dkdv_kernel(const AttnArgs a) {
   }
   const float slope = a.alibi ? a.alibi[h] : 0.f;
   // queries i that see key j: lo(i) <= j <= hi(i)
-  const int i_lo = queries_lo(a, j), i_hi = queries_hi(a, j);
+  const int i_lo = queries_lo(a, j), i_hi = queries_hi(a, j, sv.len);
   for (int i = i_lo; i <= i_hi; ++i) {
     const T* qr = qb + i * a.sq.n;
     const T* dor = dob + i * a.sdo.n;
@@ -142,8 +144,8 @@ __global__ void __launch_bounds__(128) simt_bwd_dkdv_kernel(const AttnArgs a) {
       dk[e] = fmaf(ds, qf[e], dk[e]);
     }
   }
-  T* dkr = static_cast<T*>(a.dk) + b * a.sdk.b + j * a.sdk.n + h * a.sdk.h;
-  T* dvr = static_cast<T*>(a.dv) + b * a.sdv.b + j * a.sdv.n + h * a.sdv.h;
+  T* dkr = row_ptr<T>(a.dk, a.sdk, sv, j, h);
+  T* dvr = row_ptr<T>(a.dv, a.sdv, sv, j, h);
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     dkr[lane + 32 * e] = from_f<T>(dk[e] * a.scale);
@@ -158,13 +160,14 @@ __global__ void __launch_bounds__(128) simt_bwd_dq_kernel(const AttnArgs a) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int i = blockIdx.x * 4 + warp;
   const int h = blockIdx.y, b = blockIdx.z;
-  if (i >= a.N) return;
-  const T* qr = static_cast<const T*>(a.q) + b * a.sq.b + i * a.sq.n + h * a.sq.h;
-  const T* dor = static_cast<const T*>(a.dout) + b * a.sdo.b + i * a.sdo.n + h * a.sdo.h;
-  const T* kb = static_cast<const T*>(a.k) + b * a.sk.b + h * a.sk.h;
-  const T* vb = static_cast<const T*>(a.v) + b * a.sv.b + h * a.sv.h;
-  const float lse_i = a.lse[(size_t(b) * a.H + h) * a.N + i];
-  const float d_i = a.dvec[(size_t(b) * a.H + h) * a.N + i];
+  const SeqView sv = seq_view(a.cu_seqlens, b, a.N, a.total);
+  if (i >= sv.len) return;
+  const T* qr = row_ptr<const T>(a.q, a.sq, sv, i, h);
+  const T* dor = row_ptr<const T>(a.dout, a.sdo, sv, i, h);
+  const T* kb = row_ptr<const T>(a.k, a.sk, sv, 0, h);
+  const T* vb = row_ptr<const T>(a.v, a.sv, sv, 0, h);
+  const float lse_i = a.lse[stat_index(a, sv, h, i)];
+  const float d_i = a.dvec[stat_index(a, sv, h, i)];
   float qf[E], df[E], dq[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -173,7 +176,7 @@ __global__ void __launch_bounds__(128) simt_bwd_dq_kernel(const AttnArgs a) {
     dq[e] = 0.f;
   }
   const float slope = a.alibi ? a.alibi[h] : 0.f;
-  const int lo = visible_lo(a, i), hi = visible_hi(a, i);
+  const int lo = visible_lo(a, i), hi = visible_hi(a, i, sv.len);
   for (int j = lo; j <= hi; ++j) {
     const T* kr = kb + j * a.sk.n;
     const T* vr = vb + j * a.sv.n;
@@ -196,7 +199,7 @@ __global__ void __launch_bounds__(128) simt_bwd_dq_kernel(const AttnArgs a) {
 #pragma unroll
     for (int e = 0; e < E; ++e) dq[e] = fmaf(ds, kf[e], dq[e]);
   }
-  T* dqr = static_cast<T*>(a.dq) + b * a.sdq.b + i * a.sdq.n + h * a.sdq.h;
+  T* dqr = row_ptr<T>(a.dq, a.sdq, sv, i, h);
 #pragma unroll
   for (int e = 0; e < E; ++e) dqr[lane + 32 * e] = from_f<T>(dq[e] * a.scale);
 }

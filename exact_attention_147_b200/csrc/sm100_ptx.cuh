@@ -13,6 +13,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "status.cuh"
+
 namespace fa2 {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -62,12 +64,6 @@ __device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-
-// Device-side error word shared by all kernels of the library (0 = OK).
-// A wait that runs past its time limit records its site code here and the
-// kernel winds down instead of spinning forever.  (The library is a single
-// translation unit, so the definition lives in this header.)
-__device__ int g_fa2_device_status = 0;
 
 // Shared abort flag of one CTA: set when any of its waits gives up, so the
 // other roles stop waiting too.

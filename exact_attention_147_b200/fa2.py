@@ -37,8 +37,10 @@ NOALLOC_MAX_DQ_FLOATS = 4 * 1024 * 1024
 
 # Every symbol include/fa2.h declares.
 EXPORTED = ("fa2_fwd", "fa2_bwd_preprocess", "fa2_bwd_workspace_size", "fa2_bwd",
-            "fa2_strerror", "fa2_device_status", "fa2_set_wait_limit_ms",
-            "fa2_kernel_launches", "fa2_bwd_noalloc")
+            "fa2_fwd_varlen", "fa2_bwd_varlen", "fa2_strerror", "fa2_device_status",
+            "fa2_set_wait_limit_ms", "fa2_kernel_launches", "fa2_bwd_noalloc")
+# Device status code of a packed call whose cu_seqlens was malformed.
+STATUS_BAD_SEQLENS = 0xF10
 
 
 class Strides(ctypes.Structure):
@@ -75,6 +77,13 @@ def load_library(path: str = LIB_PATH):
     lib.fa2_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
                             i, i, i, i, i, s, s, s, s, s, s, s, f, i, i, i, vp, f, u64, i, vp]
     lib.fa2_bwd.restype = i
+    lib.fa2_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, s, s, s, s, f, i, i, i,
+                                   vp, f, u64, vp]
+    lib.fa2_fwd_varlen.restype = i
+    lib.fa2_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp,
+                                   i, i, i, i, i, i, s, s, s, s, s, s, s, f, i, i, i, vp, f, u64,
+                                   i, vp]
+    lib.fa2_bwd_varlen.restype = i
     lib.fa2_strerror.argtypes = [i]
     lib.fa2_strerror.restype = ctypes.c_char_p
     lib.fa2_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), i]
@@ -115,6 +124,20 @@ def _strides(t: torch.Tensor) -> Strides:
     return Strides(t.stride(0), t.stride(1), t.stride(2))
 
 
+def _packed_strides(t: torch.Tensor) -> Strides:
+    if t.dim() != 3:
+        raise ValueError("expected a packed [total, heads, head_dim] tensor")
+    if t.stride(2) != 1:
+        raise ValueError("head_dim must be contiguous (stride 1)")
+    return Strides(0, t.stride(0), t.stride(1))
+
+
+def _seqlens(cu_seqlens: torch.Tensor) -> torch.Tensor:
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor of B + 1 offsets")
+    return cu_seqlens.contiguous()
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -153,7 +176,16 @@ def fwd(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1),
 
 
 def bwd_preprocess(out, dout, D=None, stream=None):
-    """D[b,h,i] = sum_c dout[b,i,h,c] * out[b,i,h,c] (fp32)."""
+    """D[b,h,i] = sum_c dout[b,i,h,c] * out[b,i,h,c] (fp32).
+
+    Packed [total, H, d] tensors give D as [H, total]."""
+    if out.dim() == 3:
+        total, H, _ = out.shape
+        if D is None:
+            D = torch.empty((H, total), dtype=torch.float32, device=out.device)
+        if total > 0:
+            bwd_preprocess(out.unsqueeze(0), dout.unsqueeze(0), D.unsqueeze(0), stream)
+        return D
     lib = load_library()
     B, N, H, d = out.shape
     if D is None:
@@ -191,6 +223,59 @@ def bwd(dout, q, k, v, lse, D, softmax_scale=None, causal=False, window_size=(-1
                      int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, int(bool(deterministic)),
                      _stream(stream))
     _check(st, "fa2_bwd")
+    return dq, dk, dv
+
+
+def fwd_varlen(q, k, v, cu_seqlens, max_seqlen, softmax_scale=None, causal=False,
+               window_size=(-1, -1), alibi_slopes=None, dropout_p=0.0, out=None, lse=None,
+               stream=None, dropout_seed=0):
+    """Forward pass of a packed batch: q, k, v are [total, H, d], sequence b
+    owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (int32, on the device).
+    Returns (out [total, H, d], lse [H, total] fp32)."""
+    lib = load_library()
+    total, H, d = q.shape
+    cu = _seqlens(cu_seqlens)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
+    c, wl, wr = _window(causal, window_size)
+    st = lib.fa2_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu),
+                            cu.numel() - 1, int(max_seqlen), total, H, d, _dtype_code(q),
+                            _packed_strides(q), _packed_strides(k), _packed_strides(v),
+                            _packed_strides(out), _scale(softmax_scale), c, wl, wr,
+                            _ptr(alibi_slopes), float(dropout_p),
+                            int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, _stream(stream))
+    _check(st, "fa2_fwd_varlen")
+    return out, lse
+
+
+def bwd_varlen(dout, q, k, v, lse, D, cu_seqlens, max_seqlen, softmax_scale=None,
+               causal=False, window_size=(-1, -1), alibi_slopes=None, dropout_p=0.0,
+               deterministic=False, dq=None, dk=None, dv=None, workspace=None, stream=None,
+               dropout_seed=0):
+    """Backward pass of a packed batch; returns (dq, dk, dv) shaped like q, k, v."""
+    lib = load_library()
+    total, H, d = q.shape
+    cu = _seqlens(cu_seqlens)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = workspace_size(1, total, H, d, q.dtype, deterministic) if total > 0 else 0
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    c, wl, wr = _window(causal, window_size)
+    st = lib.fa2_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(D), _ptr(dq),
+                            _ptr(dk), _ptr(dv), _ptr(workspace), wbytes, _ptr(cu),
+                            cu.numel() - 1, int(max_seqlen), total, H, d, _dtype_code(q),
+                            _packed_strides(q), _packed_strides(k), _packed_strides(v),
+                            _packed_strides(dout), _packed_strides(dq), _packed_strides(dk),
+                            _packed_strides(dv), _scale(softmax_scale), c, wl, wr,
+                            _ptr(alibi_slopes), float(dropout_p),
+                            int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, int(bool(deterministic)),
+                            _stream(stream))
+    _check(st, "fa2_bwd_varlen")
     return dq, dk, dv
 
 
@@ -240,3 +325,36 @@ def flash_attention_v2(q, k, v, dropout_p=0.0, softmax_scale=None, causal=False,
     """Exact attention with autograd support; q, k, v are [B, N, H, d]."""
     return _Fa2Function.apply(q, k, v, dropout_p, softmax_scale, causal, window_size,
                               alibi_slopes, deterministic)
+
+
+class _Fa2VarlenFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, cu_seqlens, max_seqlen, dropout_p, softmax_scale, causal,
+                window_size, alibi_slopes, deterministic):
+        seed = int(torch.randint(0, 2**63 - 1, (1,)).item()) if dropout_p > 0 else 0
+        out, lse = fwd_varlen(q, k, v, cu_seqlens, max_seqlen, softmax_scale, causal,
+                              window_size, alibi_slopes, dropout_p, dropout_seed=seed)
+        ctx.save_for_backward(q, k, v, out, lse, cu_seqlens, alibi_slopes)
+        ctx.opts = (max_seqlen, dropout_p, softmax_scale, causal, window_size, deterministic,
+                    seed)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse, cu_seqlens, alibi_slopes = ctx.saved_tensors
+        max_seqlen, dropout_p, softmax_scale, causal, window_size, deterministic, seed = ctx.opts
+        dout = dout if dout.stride(-1) == 1 else dout.contiguous()
+        D = bwd_preprocess(out, dout)
+        dq, dk, dv = bwd_varlen(dout, q, k, v, lse, D, cu_seqlens, max_seqlen, softmax_scale,
+                                causal, window_size, alibi_slopes, dropout_p, deterministic,
+                                dropout_seed=seed)
+        return dq, dk, dv, None, None, None, None, None, None, None, None
+
+
+def flash_attention_v2_varlen(q, k, v, cu_seqlens, max_seqlen, dropout_p=0.0,
+                              softmax_scale=None, causal=False, window_size=(-1, -1),
+                              alibi_slopes=None, deterministic=False):
+    """Exact attention of a packed batch with autograd support: q, k, v are
+    [total, H, d] and sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1."""
+    return _Fa2VarlenFunction.apply(q, k, v, cu_seqlens, max_seqlen, dropout_p, softmax_scale,
+                                    causal, window_size, alibi_slopes, deterministic)

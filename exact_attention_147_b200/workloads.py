@@ -9,6 +9,10 @@ q, k, v and dO as float32 N(0, 1) tensors of shape [B, N, H, d]; each is
 multiplied by its standard deviation and then cast to the compute dtype
 (bf16 or fp32).  The values the GPU receives are therefore exactly the
 values the oracle widens to float64.
+
+Packed (variable-length) workloads list their sequence lengths; their
+tensors are drawn the same way with shape [total, H, d], total = sum of the
+lengths, and ``cu_seqlens`` holds the running sums (int32).
 """
 
 from __future__ import annotations
@@ -41,6 +45,22 @@ class Workload:
     do_std: float = 1.0
     scale: float | None = None
     tags: tuple = field(default_factory=tuple)
+    lengths: tuple = ()        # packed workloads: one length per sequence
+
+    @property
+    def packed(self) -> bool:
+        return len(self.lengths) > 0
+
+    @property
+    def total(self) -> int:
+        return sum(self.lengths) if self.packed else self.B * self.N
+
+    def cu_seqlens(self, device="cpu"):
+        """Running sums [0, L_0, L_0 + L_1, ...] as int32."""
+        cu = [0]
+        for n in self.lengths:
+            cu.append(cu[-1] + n)
+        return torch.tensor(cu, dtype=torch.int32, device=device)
 
     @property
     def softmax_scale(self) -> float:
@@ -65,7 +85,7 @@ def make_inputs(w: Workload, device: str | torch.device = "cpu",
     """Draw (q, k, v, dO) for workload ``w`` (see the module docstring)."""
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed)
-    shape = (w.B, w.N, w.H, w.d)
+    shape = (w.total, w.H, w.d) if w.packed else (w.B, w.N, w.H, w.d)
     out = []
     stds = (w.q_std, w.k_std, w.v_std, w.do_std)
     for i, std in enumerate(stds):
@@ -122,6 +142,34 @@ def alibi_det() -> Workload:
     """B=4, H=16, N=4096, d=128, causal, ALiBi, deterministic backward."""
     return Workload(name="alibi-det-b4-h16-n4096", B=4, N=4096, H=16, d=128,
                     causal=True, alibi=True, deterministic=True, seed=4)
+
+
+def packed(name: str, lengths, H: int, d: int, **kw) -> Workload:
+    """A packed batch of sequences of the given lengths (B = their number,
+    N = the longest, which sizes the grids)."""
+    lengths = tuple(int(n) for n in lengths)
+    return Workload(name=name, B=len(lengths), N=max(max(lengths), 1), H=H, d=d,
+                    lengths=lengths, **kw)
+
+
+def length_mix(total: int, lo: int, hi: int, seed: int):
+    """Sequence lengths drawn uniformly from [lo, hi] (seeded) until they sum
+    to ``total`` (the last one is cut to fit)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    out, left = [], total
+    while left > 0:
+        n = int(torch.randint(lo, hi + 1, (1,), generator=g).item())
+        out.append(min(n, left))
+        left -= out[-1]
+    return tuple(out)
+
+
+def packed_mix(causal: bool = False, total: int = 32768) -> Workload:
+    """``total`` tokens in sequences of 128 to 4096 tokens (uniform, seed 5),
+    H=16, d=128, bf16."""
+    return packed(f"packed-mix-{total // 1024}k-h16-d128" + ("-causal" if causal else ""),
+                  length_mix(total, 128, 4096, seed=5), H=16, d=128, causal=causal, seed=5)
 
 
 def all_parity_workloads():

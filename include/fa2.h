@@ -43,7 +43,9 @@
  *    unimplemented combination returns FA2_ERR_UNSUPPORTED; a CUDA error at
  *    launch returns FA2_ERR_CUDA.
  *  - Supported shapes: d in {64, 128}; 1 <= N; B, H >= 1; the key/value
- *    sequence has the same length and head count as the queries.
+ *    sequence has the same length and head count as the queries.  Packed
+ *    batches of sequences of different lengths have their own entry points
+ *    (fa2_fwd_varlen, fa2_bwd_varlen) with a [total, H, d] layout.
  *  - dtype FA2_BF16: bf16 inputs/outputs, fp32 accumulation on the tensor
  *    cores.  dtype FA2_F32: fp32 inputs/outputs with full fp32 arithmetic
  *    (CUDA cores), for checks at 1e-4.
@@ -68,7 +70,8 @@ typedef enum {
   FA2_ERR_INVALID_ARG = 1,     /* a pointer, shape, stride or option is invalid */
   FA2_ERR_UNSUPPORTED = 2,     /* valid, but not implemented (e.g. dropout_p != 0) */
   FA2_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed */
-  FA2_ERR_DEVICE_TIMEOUT = 4,  /* a kernel gave up a bounded wait (see fa2_device_status) */
+  FA2_ERR_DEVICE_TIMEOUT = 4,  /* a kernel gave up a bounded wait or met malformed
+                                  cu_seqlens (see fa2_device_status) */
   FA2_ERR_SCRATCH_LIMIT = 5    /* problem too large for fa2_bwd_noalloc's fixed scratch */
 } fa2_status;
 
@@ -168,6 +171,58 @@ fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout
                    int deterministic, void* stream);
 
 /*
+ * Packed variable-length batches ("dynamic sequence support", named as
+ * future work in §6 of the "FlashAttention v2" article): B independent
+ * sequences of different lengths stored back to back, with no padding rows.
+ *
+ *   cu_seqlens    DEVICE int32 [B + 1]: sequence b owns tensor rows
+ *                 [cu_seqlens[b], cu_seqlens[b + 1]); cu_seqlens[0] = 0,
+ *                 non-decreasing, cu_seqlens[B] = total.  A length may be 0.
+ *   max_seqlen    an upper bound on every length (>= 1); it sizes the grids,
+ *                 so a tight bound wastes least.
+ *   total         number of rows of every tensor (>= 0; 0 returns FA2_OK and
+ *                 launches nothing).
+ *   q, k, v, o, dout, dq, dk, dv
+ *                 [total, H, d]; only the n (row) and h strides of each
+ *                 fa2_strides value are used, with the alignment rules above.
+ *   lse, D        dense fp32 [H, total] (row statistics of row r of head h at
+ *                 h * total + r).  D comes from fa2_bwd_preprocess called with
+ *                 B = 1, N = total on the same [total, H, d] tensors.
+ *   workspace     fa2_bwd_workspace_size(1, total, H, d, dtype, deterministic)
+ *                 bytes, 256-byte aligned.
+ *
+ * Every other argument means what it means for fa2_fwd / fa2_bwd.  Each
+ * sequence is attended to on its own, as if it were the only one of a padded
+ * call at batch index b: masks, ALiBi distances and the dropout counter use
+ * positions 0 .. len_b - 1 inside the sequence, and the dropout counter's
+ * batch field is the sequence index b.
+ *
+ * cu_seqlens lives on the device and is not read on the host.  Offsets
+ * outside [0, total], decreasing offsets and lengths above max_seqlen are
+ * clamped by the kernels (no access leaves the tensors) and recorded as code
+ * 0xF10 in the device status word (fa2_device_status); the results of such
+ * a call are unspecified.
+ */
+fa2_status fa2_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const int32_t* cu_seqlens, int B, int max_seqlen, int total,
+                          int H, int d, fa2_dtype dtype,
+                          fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides so,
+                          float softmax_scale, int causal, int window_left, int window_right,
+                          const float* alibi_slopes, float dropout_p,
+                          unsigned long long dropout_seed, void* stream);
+
+fa2_status fa2_bwd_varlen(const void* q, const void* k, const void* v, const void* dout,
+                          const float* lse, const float* D, void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes,
+                          const int32_t* cu_seqlens, int B, int max_seqlen, int total,
+                          int H, int d, fa2_dtype dtype,
+                          fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides sdo,
+                          fa2_strides sdq, fa2_strides sdk, fa2_strides sdv,
+                          float softmax_scale, int causal, int window_left, int window_right,
+                          const float* alibi_slopes, float dropout_p,
+                          unsigned long long dropout_seed, int deterministic, void* stream);
+
+/*
  * fa2_bwd_noalloc: the bf16 backward pass without any caller-provided or
  * library-allocated workspace.  (No counterpart in the paper: this is an
  * interface convenience, not part of the method.)
@@ -214,9 +269,10 @@ const char* fa2_strerror(fa2_status status);
 /*
  * Reads (and, if `clear` is nonzero, resets) the device status word of the
  * current device.  Synchronises the device.  *code receives 0 if no kernel
- * has given up a bounded wait since the last clear, else the code of the
- * first wait that did.  Returns FA2_ERR_DEVICE_TIMEOUT when *code != 0,
- * FA2_OK otherwise, FA2_ERR_CUDA on a CUDA error.
+ * has given up a bounded wait or met malformed cu_seqlens (code 0xF10)
+ * since the last clear, else the code of the first such event.  Returns
+ * FA2_ERR_DEVICE_TIMEOUT when *code != 0, FA2_OK otherwise, FA2_ERR_CUDA on
+ * a CUDA error.
  */
 fa2_status fa2_device_status(int* code, int clear);
 

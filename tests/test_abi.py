@@ -104,3 +104,49 @@ def test_workspace_size(lib):
 def test_wait_limit(lib):
     assert lib.fa2_set_wait_limit_ms(0) == F.FA2_ERR_INVALID_ARG
     assert lib.fa2_set_wait_limit_ms(1000) == F.FA2_OK
+
+
+# ----------------------------------------------------------------- packed batches
+CU = ctypes.c_void_p(0x700000)          # fake, 4-byte aligned device offsets
+SP = F.Strides(0, 16 * 128, 128)        # [total, H=16, d=128] packed strides
+
+
+def call_fwd_varlen(lib, **kw):
+    a = dict(q=P, k=P, v=P, o=ctypes.c_void_p(0x200000), lse=P, cu=CU, B=3, max_seqlen=512,
+             total=1000, H=16, d=128, dtype=F.FA2_BF16, s=SP, dropout=0.0)
+    a.update(kw)
+    return lib.fa2_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu"], a["B"],
+                              a["max_seqlen"], a["total"], a["H"], a["d"], a["dtype"], a["s"],
+                              a["s"], a["s"], a["s"], 0.0, 0, -1, -1, None, a["dropout"], 0, None)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(cu=None), dict(cu=ctypes.c_void_p(0x700002)), dict(max_seqlen=0), dict(total=-1),
+    dict(B=0), dict(d=96), dict(q=None), dict(s=F.Strides(0, 12, 128)), dict(o=P),
+    dict(dropout=1.0), dict(s=F.Strides(0, 1 << 37, 128)),
+])
+def test_fwd_varlen_rejects_invalid(lib, bad):
+    assert call_fwd_varlen(lib, **bad) == F.FA2_ERR_INVALID_ARG
+
+
+def test_varlen_empty_batch_launches_nothing(lib):
+    before = lib.fa2_kernel_launches()
+    assert call_fwd_varlen(lib, total=0, q=None, k=None, v=None, o=None, lse=None) == F.FA2_OK
+    assert lib.fa2_kernel_launches() == before
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_valid_varlen_call_without_device_is_cuda_error(lib):
+    assert call_fwd_varlen(lib) == F.FA2_ERR_CUDA
+
+
+def test_bwd_varlen_checks_its_workspace(lib):
+    need = lib.fa2_bwd_workspace_size(1, 1000, 16, 128, F.FA2_BF16, 0)
+    assert need == 1000 * 16 * 128 * 4
+    args = [P, P, P, P, P, P, ctypes.c_void_p(0x300000), ctypes.c_void_p(0x400000),
+            ctypes.c_void_p(0x500000), ctypes.c_void_p(0x600000), need - 1, CU, 3, 512, 1000,
+            16, 128, F.FA2_BF16] + [SP] * 7 + [0.0, 0, -1, -1, None, 0.0, 0, 0, None]
+    assert lib.fa2_bwd_varlen(*args) == F.FA2_ERR_INVALID_ARG
+    args[11] = None                     # no cu_seqlens
+    args[10] = need
+    assert lib.fa2_bwd_varlen(*args) == F.FA2_ERR_INVALID_ARG
