@@ -54,8 +54,9 @@ def load_peaks():
 
 # ------------------------------------------------------------------ traffic
 KERNEL_SOURCES = {
-    "fa2_fwd": ["sm100_ptx.cuh", "attn_common.cuh", "fwd_sm100.cuh"],
-    "fa2_bwd": ["sm100_ptx.cuh", "attn_common.cuh", "bwd_sm100.cuh", "fwd_sm100.cuh"],
+    "fa2_fwd": ["sm100_ptx.cuh", "status.cuh", "philox.cuh", "attn_common.cuh", "fwd_sm100.cuh"],
+    "fa2_bwd": ["sm100_ptx.cuh", "status.cuh", "philox.cuh", "attn_common.cuh", "bwd_sm100.cuh",
+                "fwd_sm100.cuh"],
 }
 
 

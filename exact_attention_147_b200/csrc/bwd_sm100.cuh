@@ -456,23 +456,25 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           if (i < lo_q || i > hi_q) pr[c] = 0.f;
         }
       }
-      // Dropout: one generator call gives the bytes of this key for four
-      // consecutive queries (output word = query mod 4, byte = key mod 4).
+      // Dropout: one generator call gives the bytes of four consecutive keys
+      // (a quad of lanes: k0 is a multiple of 128) for four consecutive
+      // queries; each lane computes one call in four and the quad trades.
       uint32_t keep_lo = 0xFFFFFFFFu, keep_hi = 0xFFFFFFFFu;
       if (DROPOUT) {
         keep_lo = keep_hi = 0u;
-        const int jb = 8 * (j & 3);
 #pragma unroll
-        for (int a = 0; a < 16; ++a) {
-          const Philox4 o = philox4x32_10(uint32_t(j >> 2), uint32_t((i0 >> 2) + a), uint32_t(h),
-                                          uint32_t(b), p.drop.seed_lo, p.drop.seed_hi);
+        for (int t16 = 0; t16 < 4; ++t16) {
+          uint32_t z[4];
+          dropout_words_col16(p.drop, b, h, j, (i0 >> 2) + 4 * t16, z);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t kept = ((o.w[e] >> jb) & 0xFFu) >= p.drop.threshold ? 1u : 0u;
-            const int c = 4 * a + e;
-            if (c < 32) keep_lo |= kept << c;
-            else keep_hi |= kept << (c - 32);
-          }
+          for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t kept = dropout_keep(z[c4], e, p.drop.threshold) ? 1u : 0u;
+              const int c = 16 * t16 + 4 * c4 + e;
+              if (c < 32) keep_lo |= kept << c;
+              else keep_hi |= kept << (c - 32);
+            }
         }
       }
       auto kept = [&](int c) {
@@ -823,13 +825,25 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
       for (int c = 0; c < 4; ++c) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_base + T_DP + c * 32, u);
+        // dropout bytes of keys kv0 + c*32 .. +31 for this row (one generator
+        // call per quad of rows and 16 keys; i0 is a multiple of 128)
+        uint32_t dw[8];
+        if (DROPOUT) {
+          uint32_t z[4];
+          dropout_words_row16(p.drop, b, h, i, ((kv0 + c * 32) >> 2), z);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dw[e] = z[e];
+          dropout_words_row16(p.drop, b, h, i, ((kv0 + c * 32) >> 2) + 4, z);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dw[4 + e] = z[e];
+        }
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           // dropout bytes of keys kv0 + c*32 + 4*e4 .. +3 for this row
           uint32_t word = 0xFFFFFFFFu;
-          if (DROPOUT) word = dropout_word_row(p.drop, b, h, i, ((kv0 + c * 32) >> 2) + e4);
+          if (DROPOUT) word = dw[e4];
 #pragma unroll
           for (int e2 = 0; e2 < 2; ++e2) {
             const int e = 2 * e4 + e2;

@@ -504,21 +504,29 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
           l3 += s[c + 3];
         }
         l_run = fmaf(l_run, alpha, (l0 + l1) + (l2 + l3));
-        if (DROPOUT) {  // l keeps the un-dropped sum; dropped probabilities leave P
-#pragma unroll
-          for (int c4 = 0; c4 < BN / 4; ++c4) {
-            const uint32_t word = dropout_word_row(p.drop, b, h, i, (kv0 >> 2) + c4);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (!dropout_keep(word, e, p.drop.threshold)) s[4 * c4 + e] = 0.f;
-          }
-        }
-        // P (bf16 pairs) over the first BN/2 columns of S.
+        // P (bf16 pairs) over the first BN/2 columns of S.  With dropout, l
+        // keeps the un-dropped sum and dropped probabilities leave P here:
+        // one generator call per quad of rows and 16 keys (the rows of a quad
+        // share i / 4: row0 is a multiple of 256), applied as 16-bit masks to
+        // the packed pairs.
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t w16[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) w16[e] = pack_bf16(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]);
+          if (DROPOUT) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t z[4];
+              dropout_words_row16(p.drop, b, h, i, (kv0 >> 2) + 8 * c + 4 * half, z);
+#pragma unroll
+              for (int g4 = 0; g4 < 4; ++g4) {
+                const uint32_t m = dropout_keep_bytes(z[g4], p.drop.threshold);
+                w16[8 * half + 2 * g4] &= __byte_perm(m, 0u, 0x1100);
+                w16[8 * half + 2 * g4 + 1] &= __byte_perm(m, 0u, 0x3322);
+              }
+            }
+          }
           tmem_st16(s_addr + c * 16, w16);
         }
         // Rescale the running output (the PV product of the previous block has

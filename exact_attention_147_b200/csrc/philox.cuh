@@ -11,8 +11,10 @@
 // key j) is byte (j mod 4) (least significant first) of output word (i mod 4)
 // of Philox4x32-10 with counter (j / 4, i / 4, h, b) and key (seed low,
 // seed high).  The element is kept iff its byte is >= t = round(256 p), and
-// kept probabilities are scaled by 256 / (256 - t).  A query row therefore
-// gets four keys per generator call and a key row four queries.
+// kept probabilities are scaled by 256 / (256 - t).  One generator call
+// covers a 4 x 4 block of (query, key) pairs; the tensor-core kernels, whose
+// threads each own one row, share every call across the four lanes that own
+// the block's four rows (quad_transpose below), so each byte drawn is used.
 #pragma once
 
 #include <cstdint>
@@ -59,6 +61,71 @@ __device__ __forceinline__ uint32_t dropout_word_row(const DropoutParams& dp, in
                                   dp.seed_hi);
   const int s = i & 3;
   return s == 0 ? o.w[0] : s == 1 ? o.w[1] : s == 2 ? o.w[2] : o.w[3];
+}
+
+// The four lanes 4q .. 4q+3 of a warp (a "quad") hold four consecutive query
+// rows (or key rows) whose counters coincide, so one generator call serves
+// the whole quad: each lane computes one call of four and the quad trades the
+// results, instead of every lane computing all four and keeping a quarter.
+//
+// quad_transpose: lane s of the quad holds x[w] = the word it prepared for
+// lane w; afterwards lane r holds z[c] = the word lane c prepared for lane r.
+// Round u sends x[(s - u) mod 4] to the lane (s - u) mod 4, which reads it
+// from lane (r + u) mod 4; z is the received words rotated into place.
+// All 32 lanes of the warp must be active.
+__device__ __forceinline__ uint32_t pick4(const uint32_t (&x)[4], int k) {
+  const uint32_t lo = (k & 1) ? x[1] : x[0];
+  const uint32_t hi = (k & 1) ? x[3] : x[2];
+  return (k & 2) ? hi : lo;
+}
+
+__device__ __forceinline__ void quad_transpose(const uint32_t (&x)[4], uint32_t (&z)[4]) {
+  const int lane = int(threadIdx.x & 31u);
+  const int s = lane & 3, base = lane & ~3;
+  uint32_t y[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint32_t v = pick4(x, (s - u) & 3);
+    y[u] = u == 0 ? v : __shfl_sync(0xffffffffu, v, base | ((s + u) & 3));
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) z[c] = pick4(y, (c - s) & 3);
+}
+
+// Random words of this lane's query row i for key groups j4_0 + c, c = 0..3
+// (16 consecutive keys starting at 4 j4_0; z[c] holds keys 4(j4_0+c) ..
+// 4(j4_0+c)+3 as bytes, least significant first).  j4_0 must be a multiple
+// of 4 and the quad must hold rows i with i mod 4 = lane mod 4.
+__device__ __forceinline__ void dropout_words_row16(const DropoutParams& dp, int b, int h, int i, int j4_0,
+                                                    uint32_t (&z)[4]) {
+  const int s = int(threadIdx.x & 3u);
+  const Philox4 o = philox4x32_10(uint32_t(j4_0 + s), uint32_t(i >> 2), uint32_t(h), uint32_t(b),
+                                  dp.seed_lo, dp.seed_hi);
+  // word w of call (j4_0 + s) belongs to row 4 (i / 4) + w, i.e. quad lane w
+  quad_transpose(o.w, z);
+}
+
+// Random bytes of this lane's key row j for query groups i4_0 + c, c = 0..3
+// (16 consecutive queries starting at 4 i4_0; z[c] holds queries
+// 4(i4_0+c) .. 4(i4_0+c)+3 as bytes, least significant first).  i4_0 must be
+// a multiple of 4 and the quad must hold keys j with j mod 4 = lane mod 4.
+__device__ __forceinline__ void dropout_words_col16(const DropoutParams& dp, int b, int h, int j, int i4_0,
+                                                    uint32_t (&z)[4]) {
+  const int s = int(threadIdx.x & 3u);
+  const Philox4 o = philox4x32_10(uint32_t(j >> 2), uint32_t(i4_0 + s), uint32_t(h), uint32_t(b),
+                                  dp.seed_lo, dp.seed_hi);
+  // byte r of every word belongs to key 4 (j / 4) + r, i.e. quad lane r:
+  // transpose the 4 x 4 bytes so that x[r] gathers byte r of words 0..3
+  const uint32_t lo01 = __byte_perm(o.w[0], o.w[1], 0x5140), hi01 = __byte_perm(o.w[0], o.w[1], 0x7362);
+  const uint32_t lo23 = __byte_perm(o.w[2], o.w[3], 0x5140), hi23 = __byte_perm(o.w[2], o.w[3], 0x7362);
+  const uint32_t x[4] = {__byte_perm(lo01, lo23, 0x5410), __byte_perm(lo01, lo23, 0x7632),
+                         __byte_perm(hi01, hi23, 0x5410), __byte_perm(hi01, hi23, 0x7632)};
+  quad_transpose(x, z);
+}
+
+// 0xFF in every byte of `word` that is kept (byte >= threshold), else 0x00.
+__device__ __forceinline__ uint32_t dropout_keep_bytes(uint32_t word, uint32_t threshold) {
+  return __vcmpgeu4(word, threshold * 0x01010101u);
 }
 
 // Byte e (0..3) of a packed word kept?
