@@ -13,6 +13,7 @@ time, so that a reader can check it against the source pages by eye.  See
 
 from .attention import (  # noqa: F401
     allowed_mask,
+    block_mask_elements,
     alibi_bias,
     head_scores,
     head_forward,

@@ -41,6 +41,12 @@ Readings taken where the pages are silent (each repeated where it applies):
 * a row with no visible key (unreachable with the shipped masks, since the
   diagonal is always visible) has O = 0, LSE = -inf and zero gradients.
 
+Block-sparse masks ("FlashAttention v2" article, §6, future work: block-
+sparse attention; the pages give no formula, so the plain reading is
+taken): a boolean block mask M of shape [ceil(N / block), ceil(N / block)]
+per head hides key j from query i unless M[i // block, j // block] is true,
+on top of the causal and window masks.  The library's block is 128.
+
 Dropout (the call's ``dropout_p``; the pages give no formula, so the plain
 reading of attention dropout is taken): after the softmax, each probability
 is kept or zeroed by a given boolean mask and kept ones are multiplied by a
@@ -88,6 +94,15 @@ def allowed_mask(rows: np.ndarray, n_keys: int, causal: bool,
     return ok
 
 
+def block_mask_elements(block_mask, rows, n_keys: int, block: int) -> np.ndarray:
+    """Boolean [len(rows), n_keys]: True where block (i // block, j // block)
+    of the block mask is set."""
+    bm = np.asarray(block_mask, dtype=bool)
+    i = np.asarray(rows, dtype=np.int64) // block
+    j = np.arange(n_keys, dtype=np.int64) // block
+    return bm[i[:, None], j[None, :]]
+
+
 def alibi_bias(rows: np.ndarray, n_keys: int, slope: float) -> np.ndarray:
     """ALiBi bias -slope * |i - j| ("FlashAttention v2" article, §5.1,
     ``alibi_slopes``; sign and |i-j| form are the reading taken)."""
@@ -98,14 +113,16 @@ def alibi_bias(rows: np.ndarray, n_keys: int, slope: float) -> np.ndarray:
 
 def head_scores(q_rows: np.ndarray, k: np.ndarray, rows: np.ndarray,
                 scale: float, causal: bool, window_left: int,
-                window_right: int, slope: float | None) -> np.ndarray:
+                window_right: int, slope: float | None,
+                block_mask=None, block: int = 128) -> np.ndarray:
     """s_ij = scale * <q_i, k_j> + bias_ij, -inf where the mask hides j."""
     s = scale * (q_rows @ k.T)
     if slope is not None:
         s = s + alibi_bias(rows, k.shape[0], slope)
-    s = np.where(allowed_mask(rows, k.shape[0], causal, window_left,
-                              window_right), s, -np.inf)
-    return s
+    ok = allowed_mask(rows, k.shape[0], causal, window_left, window_right)
+    if block_mask is not None:
+        ok &= block_mask_elements(block_mask, rows, k.shape[0], block)
+    return np.where(ok, s, -np.inf)
 
 
 def _softmax_rows(s: np.ndarray):
@@ -128,12 +145,13 @@ def head_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
                  causal: bool = False, window_left: int = -1,
                  window_right: int = -1, slope: float | None = None,
                  rows: np.ndarray | None = None, keep=None,
-                 keep_scale: float = 1.0):
+                 keep_scale: float = 1.0, block_mask=None, block: int = 128):
     """One head: q [Nq_rows, d] (the rows listed in ``rows``), k, v [N, d].
 
     ``keep`` (optional): boolean [len(rows), N] dropout mask, applied to P
-    with ``keep_scale``.  Returns (O [rows, d], LSE [rows]) with
-    LSE = M + ln(l) of the un-dropped scores.
+    with ``keep_scale``.  ``block_mask`` (optional): boolean block mask of
+    this head (see the module docstring).  Returns (O [rows, d], LSE [rows])
+    with LSE = M + ln(l) of the un-dropped scores.
     """
     n = k.shape[0]
     if rows is None:
@@ -145,7 +163,7 @@ def head_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
     for r0 in range(0, rows.shape[0], chunk):
         rr = rows[r0:r0 + chunk]
         s = head_scores(q[r0:r0 + chunk], k, rr, scale, causal, window_left,
-                        window_right, slope)
+                        window_right, slope, block_mask, block)
         p, m, l = _softmax_rows(s)
         if keep is not None:
             p = p * (keep[r0:r0 + chunk] * keep_scale)
@@ -160,7 +178,7 @@ def head_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
                   do: np.ndarray, scale: float, causal: bool = False,
                   window_left: int = -1, window_right: int = -1,
                   slope: float | None = None, keep=None,
-                  keep_scale: float = 1.0):
+                  keep_scale: float = 1.0, block_mask=None, block: int = 128):
     """Textbook gradients for one head (q, k, v, do are [N, d]).
 
     The probabilities are recomputed from the inputs, as in the explainer's
@@ -176,7 +194,7 @@ def head_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     for r0 in range(0, n, chunk):
         rr = np.arange(r0, min(n, r0 + chunk))
         s = head_scores(q[rr], k, rr, scale, causal, window_left,
-                        window_right, slope)
+                        window_right, slope, block_mask, block)
         p, _, _ = _softmax_rows(s)
         mk = 1.0 if keep is None else keep[rr] * keep_scale
         pd = p * mk                            # dropped probabilities
@@ -198,9 +216,11 @@ def _slope(alibi_slopes, h):
 
 def attention_forward(q, k, v, scale: float, causal: bool = False,
                       window_left: int = -1, window_right: int = -1,
-                      alibi_slopes=None, heads=None):
+                      alibi_slopes=None, heads=None, block_mask=None,
+                      block: int = 128):
     """O [B,N,H,d] and LSE [B,H,N] for every (b, h), or only for the
-    (b, h) pairs listed in ``heads`` (other entries are left NaN)."""
+    (b, h) pairs listed in ``heads`` (other entries are left NaN).
+    ``block_mask``: optional boolean [B, H, nq_blocks, nk_blocks]."""
     q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
     b_, n, h_, d = q.shape
     o = np.full((b_, n, h_, v.shape[3]), np.nan)
@@ -210,7 +230,9 @@ def attention_forward(q, k, v, scale: float, causal: bool = False,
     for b, h in pairs:
         o[b, :, h], lse[b, h] = head_forward(
             q[b, :, h], k[b, :, h], v[b, :, h], scale, causal, window_left,
-            window_right, _slope(alibi_slopes, h))
+            window_right, _slope(alibi_slopes, h),
+            block_mask=None if block_mask is None else block_mask[b][h],
+            block=block)
     return o, lse
 
 
@@ -230,7 +252,8 @@ def attention_forward_rows(q, k, v, b: int, h: int, rows, scale: float,
 
 def attention_backward(q, k, v, do, scale: float, causal: bool = False,
                        window_left: int = -1, window_right: int = -1,
-                       alibi_slopes=None, heads=None):
+                       alibi_slopes=None, heads=None, block_mask=None,
+                       block: int = 128):
     """dq, dk, dv [B,N,H,d] and D [B,H,N] (all heads, or those in ``heads``;
     other entries are left NaN)."""
     q, k, v, do = (np.asarray(t, dtype=np.float64) for t in (q, k, v, do))
@@ -244,7 +267,9 @@ def attention_backward(q, k, v, do, scale: float, causal: bool = False,
     for b, h in pairs:
         dq[b, :, h], dk[b, :, h], dv[b, :, h], dvec[b, h] = head_backward(
             q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h], scale, causal,
-            window_left, window_right, _slope(alibi_slopes, h))
+            window_left, window_right, _slope(alibi_slopes, h),
+            block_mask=None if block_mask is None else block_mask[b][h],
+            block=block)
     return dq, dk, dv, dvec
 
 
