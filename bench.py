@@ -393,6 +393,7 @@ def run_gpu(args):
         line["by_n"] = run_sweep(F, W, args, full=args.sweep)
         line["dropout"] = run_dropout(F, W)
         line["packed"] = run_packed(F, W)
+        line["blocksparse"] = run_blocksparse(F, W)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -498,6 +499,36 @@ def run_packed(F, W):
         del q, k, v, do, out, lse, D, dq, dk, dv, ws, qp, kp, vp, dop, op_, lp, Dp, gp, wsp
         torch.cuda.empty_cache()
     return res
+
+
+def run_blocksparse(F, W):
+    """The bench workload (B=8 H=16 N=2048 d=128) with a local + global
+    block mask: a band of 3 blocks around the diagonal plus the first block
+    column (60 of 256 blocks kept).  TFLOP/s count the kept blocks only
+    (4 * 128 * 128 * d FLOPs each, forward); the dense times are for the
+    whole 2048 x 2048 product."""
+    import torch
+    w = W.mid(False)
+    nb = (w.N + 127) // 128
+    qb = torch.arange(nb)[:, None]
+    kb = torch.arange(nb)[None, :]
+    one = (((qb - kb).abs() <= 1) | (kb == 0)).to(torch.uint8)
+    mask = one.cuda()[None, None].expand(w.B, w.H, nb, nb)
+    kept = int(one.sum())
+    q, k, v, do = W.make_inputs(w, "cuda")
+    out, lse = F.fwd_blocksparse(q, k, v, mask)
+    D = F.bwd_preprocess(out, do)
+    dq, dk, dv = F.bwd_blocksparse(do, q, k, v, lse, D, mask)
+    ws = torch.empty(F.workspace_size(w.B, w.N, w.H, w.d, torch.bfloat16), dtype=torch.uint8,
+                     device="cuda")
+    tf, tb = _time_pair(
+        lambda: F.fwd_blocksparse(q, k, v, mask, out=out, lse=lse),
+        lambda: F.bwd_blocksparse(do, q, k, v, lse, D, mask, dq=dq, dk=dk, dv=dv, workspace=ws))
+    ff = 4.0 * 128 * 128 * w.d * kept * w.B * w.H
+    return {"workload": "B=8 H=16 N=2048 d=128, band 3 + first column", "blocks_kept": kept,
+            "blocks": nb * nb, "fwd_ms": round(tf, 4),
+            "fwd_tflops": round(ff / (tf * 1e-3) / 1e12, 1), "bwd_ms": round(tb, 4),
+            "bwd_tflops": round(2.5 * ff / (tb * 1e-3) / 1e12, 1)}
 
 
 def run_sweep(F, W, args, full=False):

@@ -9,6 +9,11 @@
 
 namespace fa2 {
 
+// Layout modes of the tensor-core kernels (template argument MODE).
+constexpr int kLayoutPadded = 0;   // [B, N, H, d]
+constexpr int kLayoutPacked = 1;   // [total, H, d] with cu_seqlens
+constexpr int kLayoutSparse = 2;   // [B, N, H, d] with a 128 x 128 block mask
+
 struct Strides {
   int64_t b, n, h;  // element strides of a [B, N, H, d] tensor (d stride 1)
 };
@@ -41,6 +46,8 @@ struct AttnArgs {
   float* dq_accum;    // fp32 [B*H, N, d] (padded) or [H, total, d] (packed) workspace
   const int* cu_seqlens;  // [B + 1] device offsets (packed) or null (padded)
   int total;          // packed: rows of the tensors; padded: unused
+  const uint8_t* block_mask;  // [B, H, nb, nb] 128 x 128 block mask (padded only) or null
+  int64_t bm_sb, bm_sh;       // its batch and head strides in elements; rows hold nb bytes
   Strides sq, sk, sv, so, sdo, sdq, sdk, sdv;
   int B, N, H, d;
   float scale;        // softmax scale
@@ -93,6 +100,13 @@ __device__ __forceinline__ T* row_ptr(P* base, const Strides& s, const SeqView& 
 __device__ __forceinline__ size_t stat_index(const AttnArgs& a, const SeqView& v, int h, int i) {
   const int rows = a.cu_seqlens ? a.total : a.N;
   return (size_t(v.bt) * a.H + h) * size_t(rows) + size_t(v.row0 + i);
+}
+
+// Block mask: may query i see key j at all?  (nb = ceil(N / 128).)
+__device__ __forceinline__ bool block_kept(const AttnArgs& a, int b, int h, int i, int j) {
+  if (a.block_mask == nullptr) return true;
+  const int64_t nb = (a.N + 127) / 128;
+  return a.block_mask[b * a.bm_sb + h * a.bm_sh + (i >> 7) * nb + (j >> 7)] != 0;
 }
 
 // Keys visible to query i of a sequence of n rows lie in [visible_lo,

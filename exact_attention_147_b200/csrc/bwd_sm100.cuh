@@ -57,6 +57,9 @@ struct BwdParams {
   const int* cu_seqlens;                 // [B+1] sequence offsets (packed) or null (padded)
   int total;                             // packed: tensor rows
   int stat_rows;                         // rows per (batch, head) of lse / D: N or total
+  const uint8_t* bmask;                  // block-sparse: [B, H, nb, nb] 128 x 128 block mask
+  long long bm_sb, bm_sh;                // its batch and head strides (elements)
+  int nb;                                // ceil(N / 128)
   int N, H, B;                           // N: the (longest) sequence length
   int wl, wr;
   int nblocks;                           // ceil(N / 128)
@@ -135,6 +138,30 @@ __device__ __forceinline__ void st_sw128_row32(uint8_t* tile, int row, int col0,
   }
 }
 
+// Block-sparse iteration: the first index after x, up to `last`, whose mask
+// byte m[index * stride] is set (`last` itself when none before it is).
+__device__ __forceinline__ int next_kept(const uint8_t* m, long long stride, int x, int last) {
+  for (++x; x < last; ++x)
+    if (m[x * stride] != 0) break;
+  return x;
+}
+
+// Kept blocks among [first, last] of a mask line: sets first to the first
+// kept one and returns their count, or leaves first alone and returns 1 when
+// none is kept (the kernel then visits one fully hidden block, which writes
+// zero gradients).
+__device__ __forceinline__ int count_kept(const uint8_t* m, long long stride, int& first, int last) {
+  int cnt = 0, f = -1;
+  for (int x = first; x <= last; ++x)
+    if (m[x * stride] != 0) {
+      if (f < 0) f = x;
+      ++cnt;
+    }
+  if (cnt == 0) return 1;
+  first = f;
+  return cnt;
+}
+
 // Writes the same 16 words straight to row `row` of a global bf16 tensor
 // (columns col0 .. col0 + 31): the output path of tiles whose last rows
 // belong to the next sequence of a packed batch, which a TMA store of the
@@ -164,9 +191,11 @@ __device__ __forceinline__ void st_global_row32(__nv_bfloat16* base, const Strid
 // adds it into the fp32 accumulator with TMA bulk reductions, which go
 // through the TMA unit rather than the load/store queues.
 // ---------------------------------------------------------------------------
-template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT, bool PACKED>
+template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT, int MODE>
 __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<HD>;
+  constexpr bool PACKED = MODE == kLayoutPacked;
+  constexpr bool SPARSE = MODE == kLayoutSparse;
   using namespace bwd_detail;
   constexpr int QS = C::Q_STAGES, DS = C::DO_STAGES;
   constexpr int NCH = HD / 64;
@@ -219,8 +248,13 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   const int k_last = min(len - 1, k0 + 127);
   const int i_lo = p.wr >= 0 ? max(0, k0 - p.wr) : 0;
   const int i_hi = p.wl >= 0 ? min(len - 1, k_last + p.wl) : len - 1;
-  const int qb_begin = i_lo / 128;
-  const int nq = i_hi / 128 - qb_begin + 1;
+  // query blocks visited: [qb_first, qb_last], only the kept ones when a
+  // block mask is given (this key block's mask column: mcol[qb * nb])
+  int qb_first = i_lo / 128;
+  const int qb_last = i_hi / 128;
+  const uint8_t* mcol = SPARSE ? p.bmask + b * p.bm_sb + h * p.bm_sh + kb : nullptr;
+  const int nq = SPARSE ? count_kept(mcol, p.nb, qb_first, qb_last) : qb_last - qb_first + 1;
+  auto next_qb = [&](int qb) { return SPARSE ? next_kept(mcol, p.nb, qb, qb_last) : qb + 1; };
   const size_t head_off = (size_t(sv.bt) * p.H + h) * (PACKED ? p.stat_rows : p.N) + sv.row0;
   const int trow = sv.row0;       // tensor row of local row 0
 
@@ -257,8 +291,9 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       }
       int issued_q = 0, issued_do = 0;
       bool ok = true;
-      for (int it = 0; it < nq && ok; ++it) {
-        const int i0 = (qb_begin + it) * 128;
+      int qb = qb_first;
+      for (int it = 0; it < nq && ok; ++it, qb = next_qb(qb)) {
+        const int i0 = (SPARSE ? qb : qb_first + it) * 128;
         const int sq = it % QS;
         // log2-scaled LSE and D of this query block, +inf / 0 past the end; loaded
         // before waiting for the slot so the latency overlaps the wait
@@ -412,8 +447,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
     float slope2 = 0.f;
     if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
     bool ok = true;
-    for (int it = 0; it < nq; ++it) {
-      const int i0 = (qb_begin + it) * 128 + cq;
+    int qb = qb_first;
+    for (int it = 0; it < nq; ++it, qb = next_qb(qb)) {
+      const int i0 = (SPARSE ? qb : qb_first + it) * 128 + cq;
+      // a fully hidden block is visited only when the mask keeps none
+      const bool hidden = SPARSE && mcol[qb * p.nb] == 0;
       const float* side = sSide + (it % QS) * 256 + cq;
       ok = wait_bar(s_full, it & 1, ab, p.wait_ns, SITE_BCOMP + 0);
       ok = __all_sync(0xffffffffu, ok);
@@ -449,11 +487,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           pr[c + 3] = ex2(x3);
         }
       }
-      if (!full) {
+      if (!full || hidden) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int i = i0 + c;
-          if (i < lo_q || i > hi_q) pr[c] = 0.f;
+          if (hidden || i < lo_q || i > hi_q) pr[c] = 0.f;
         }
       }
       // Dropout: one generator call gives the bytes of four consecutive keys
@@ -583,8 +621,9 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       const int q = (warp % 4) * 32 + lane;
       const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
       const int bh = sv.bt * p.H + h;
-      for (int it = 0; it < nq; ++it) {
-        const int i0 = (qb_begin + it) * 128;
+      int qb = qb_first;
+      for (int it = 0; it < nq; ++it, qb = next_qb(qb)) {
+        const int i0 = (SPARSE ? qb : qb_first + it) * 128;
         bool ok = wait_bar(dq_full, it & 1, ab, p.wait_ns, SITE_BRED);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
@@ -637,9 +676,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
 // ---------------------------------------------------------------------------
 // Kernel 2: dQ by an ordered walk over key blocks (deterministic mode)
 // ---------------------------------------------------------------------------
-template <int HD, bool ALIBI, bool DROPOUT, bool PACKED>
+template <int HD, bool ALIBI, bool DROPOUT, int MODE>
 __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_constant__ BwdParams p) {
   using C = DqCfg<HD>;
+  constexpr bool PACKED = MODE == kLayoutPacked;
+  constexpr bool SPARSE = MODE == kLayoutSparse;
   using namespace bwd_detail;
   constexpr int SLOTS = C::SLOTS;
   constexpr int NCH = HD / 64;
@@ -681,8 +722,13 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
   const int i_last = min(len - 1, i0 + 127);
   const int kv_lo = p.wl >= 0 ? max(0, i0 - p.wl) : 0;
   const int kv_hi = p.wr >= 0 ? min(len - 1, i_last + p.wr) : len - 1;
-  const int kb_begin = kv_lo / 128;
-  const int nk = kv_hi / 128 - kb_begin + 1;
+  // key blocks visited: [kb_first, kb_last], only the kept ones when a block
+  // mask is given (this query block's mask row)
+  int kb_first = kv_lo / 128;
+  const int kb_last = kv_hi / 128;
+  const uint8_t* mrow = SPARSE ? p.bmask + b * p.bm_sb + h * p.bm_sh + (long long)qb * p.nb : nullptr;
+  const int nk = SPARSE ? count_kept(mrow, 1, kb_first, kb_last) : kb_last - kb_first + 1;
+  auto next_kb = [&](int kb) { return SPARSE ? next_kept(mrow, 1, kb, kb_last) : kb + 1; };
   const size_t head_off = (size_t(sv.bt) * p.H + h) * (PACKED ? p.stat_rows : p.N) + sv.row0;
   const int trow = sv.row0;       // tensor row of local row 0
 
@@ -713,8 +759,9 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
       }
       int n = 0;
       bool ok = true;
-      for (int it = 0; it < nk && ok; ++it) {
-        const int kv0 = trow + (kb_begin + it) * 128;
+      int kb = kb_first;
+      for (int it = 0; it < nk && ok; ++it, kb = next_kb(kb)) {
+        const int kv0 = trow + (SPARSE ? kb : kb_first + it) * 128;
         for (int which = 0; which < 2; ++which, ++n) {
           const int s = n % SLOTS;
           if (!wait_bar(slot_empty(s), ((n / SLOTS) & 1) ^ 1, ab, p.wait_ns, SITE_QPROD)) {
@@ -788,8 +835,11 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
     }
     if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
     bool ok = true;
-    for (int it = 0; it < nk; ++it) {
-      const int kv0 = (kb_begin + it) * 128;
+    int kb = kb_first;
+    for (int it = 0; it < nk; ++it, kb = next_kb(kb)) {
+      const int kv0 = (SPARSE ? kb : kb_first + it) * 128;
+      // a fully hidden block is visited only when the mask keeps none
+      const bool hidden = SPARSE && mrow[kb] == 0;
       ok = wait_bar(s_full, it & 1, ab, p.wait_ns, SITE_QCOMP + 0);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -810,11 +860,11 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
         if (ALIBI) x = fmaf(slope2, fabsf(fi - float(c)), x);
         pr[c] = ex2(x);
       }
-      if (!(kv0 >= lo && kv0 + 127 <= hi)) {
+      if (hidden || !(kv0 >= lo && kv0 + 127 <= hi)) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
           const int j = kv0 + c;
-          if (j < lo || j > hi) pr[c] = 0.f;
+          if (hidden || j < lo || j > hi) pr[c] = 0.f;
         }
       }
       ok = wait_bar(dp_full, it & 1, ab, p.wait_ns, SITE_QCOMP + 1);

@@ -231,7 +231,7 @@ fa2_status dispatch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa
                               const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
                               int causal_order, cudaStream_t st);
 
-template <int HD, bool ALIBI, bool DROPOUT, bool PACKED>
+template <int HD, bool ALIBI, bool DROPOUT, int MODE>
 fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
                             const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
                             int causal_order, cudaStream_t st) {
@@ -261,8 +261,12 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.wait_ns = g_wait_ns.load();
   p.drop = a.drop;
-  if (PACKED) FA2_TRY(sched_counters(dev, &p.sched));
-  auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, PACKED>;
+  p.bmask = a.block_mask;
+  p.bm_sb = a.bm_sb;
+  p.bm_sh = a.bm_sh;
+  p.nb = (a.N + 127) / 128;
+  if (MODE != kLayoutPadded) FA2_TRY(sched_counters(dev, &p.sched));
+  auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, MODE>;
   constexpr int smem = FwdCfg<HD>::SMEM_BYTES;
   FA2_TRY(ensure_smem(kern, smem, dev, mask));
   // persistent grid: one CTA per SM (shared memory and TMEM allow one)
@@ -271,7 +275,7 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   return launched(1);
 }
 
-template <int HD, bool ALIBI, bool DROPOUT, bool PACKED>
+template <int HD, bool ALIBI, bool DROPOUT, int MODE>
 fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
                             const fa2_strides& sv, const fa2_strides& sdo, const fa2_strides& sdq,
                             const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
@@ -301,6 +305,10 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.cu_seqlens = a.cu_seqlens;
   p.total = a.total;
   p.stat_rows = ms.rows;
+  p.bmask = a.block_mask;
+  p.bm_sb = a.bm_sb;
+  p.bm_sh = a.bm_sh;
+  p.nb = (a.N + 127) / 128;
   p.N = a.N;
   p.H = a.H;
   p.B = a.B;
@@ -322,8 +330,8 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   // forever.  Refuse to launch otherwise.
   {
     cudaFuncAttributes fa;
-    auto k1c = deterministic ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, PACKED>
-                             : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, PACKED>;
+    auto k1c = deterministic ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, MODE>
+                             : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE>;
     if (cudaFuncGetAttributes(&fa, k1c) != cudaSuccess) return FA2_ERR_CUDA;
     if (fa.numRegs < BwdCfg<HD>::REGS_AT_LAUNCH) return FA2_ERR_UNSUPPORTED;
   }
@@ -332,7 +340,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
     const unsigned zgrid = unsigned(std::min<long long>((n4 + 255) / 256, 148 * 16));
     zero_f32x4_kernel<<<zgrid, 256, 0, st>>>(reinterpret_cast<float4*>(a.dq_accum), n4);
     FA2_TRY(launched(1));
-    auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, PACKED>;
+    auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE>;
     FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv));
     k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
     FA2_TRY(launched(1));
@@ -345,11 +353,11 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
     dq_convert_kernel<HD><<<unsigned((rows + per_block - 1) / per_block), 256, 0, st>>>(c);
     return launched(1);
   }
-  auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, PACKED>;
+  auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, MODE>;
   FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv_nodq));
   k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
   FA2_TRY(launched(1));
-  auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI, DROPOUT, PACKED>;
+  auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI, DROPOUT, MODE>;
   constexpr int smem2 = DqCfg<HD>::SMEM_BYTES;
   FA2_TRY(ensure_smem(k2, smem2, dev, mask_dq));
   k2<<<grid, DqCfg<HD>::THREADS, smem2, st>>>(p);
@@ -372,12 +380,15 @@ fa2_status dispatch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa
                               const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
                               int causal_order, cudaStream_t st) {
   return static_bools(
-      [&](auto alibi, auto dropout, auto packed) {
-        return launch_fwd_sm100<HD, decltype(alibi)::value, decltype(dropout)::value,
-                                decltype(packed)::value>(a, sq, sk, sv, so, dev, sm_count,
-                                                         causal_order, st);
+      [&](auto alibi, auto dropout) {
+        constexpr bool A = decltype(alibi)::value, D = decltype(dropout)::value;
+        if (a.cu_seqlens)
+          return launch_fwd_sm100<HD, A, D, kLayoutPacked>(a, sq, sk, sv, so, dev, sm_count, causal_order, st);
+        if (a.block_mask)
+          return launch_fwd_sm100<HD, A, D, kLayoutSparse>(a, sq, sk, sv, so, dev, sm_count, causal_order, st);
+        return launch_fwd_sm100<HD, A, D, kLayoutPadded>(a, sq, sk, sv, so, dev, sm_count, causal_order, st);
       },
-      a.alibi != nullptr, a.dropout != 0, a.cu_seqlens != nullptr);
+      a.alibi != nullptr, a.dropout != 0);
 }
 
 template <int HD>
@@ -386,12 +397,18 @@ fa2_status dispatch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa
                               const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
                               int dev, cudaStream_t st) {
   return static_bools(
-      [&](auto alibi, auto dropout, auto packed) {
-        return launch_bwd_sm100<HD, decltype(alibi)::value, decltype(dropout)::value,
-                                decltype(packed)::value>(a, sq, sk, sv, sdo, sdq, sdk, sdv,
+      [&](auto alibi, auto dropout) {
+        constexpr bool A = decltype(alibi)::value, D = decltype(dropout)::value;
+        if (a.cu_seqlens)
+          return launch_bwd_sm100<HD, A, D, kLayoutPacked>(a, sq, sk, sv, sdo, sdq, sdk, sdv,
+                                                           deterministic, dev, st);
+        if (a.block_mask)
+          return launch_bwd_sm100<HD, A, D, kLayoutSparse>(a, sq, sk, sv, sdo, sdq, sdk, sdv,
+                                                           deterministic, dev, st);
+        return launch_bwd_sm100<HD, A, D, kLayoutPadded>(a, sq, sk, sv, sdo, sdq, sdk, sdv,
                                                          deterministic, dev, st);
       },
-      a.alibi != nullptr, a.dropout != 0, a.cu_seqlens != nullptr);
+      a.alibi != nullptr, a.dropout != 0);
 }
 
 // ----------------------------------------------------------------- packed checks
@@ -408,6 +425,13 @@ fa2_status check_packed_tensor(const void* p, fa2_strides s, fa2_dtype dtype, in
   if (s.n >= 1 && int64_t(total) * s.n >= lim) return FA2_ERR_INVALID_ARG;
   s.b = s.n;  // checked like the others, then ignored
   return check_tensor(p, s, dtype);
+}
+
+// Block mask: device bytes, batch/head strides >= 0 (0 shares one mask).
+fa2_status check_block_mask(const uint8_t* m, int64_t sb, int64_t sh) {
+  if (m == nullptr || sb < 0 || sh < 0) return FA2_ERR_INVALID_ARG;
+  if (sb >= (int64_t(1) << 40) || sh >= (int64_t(1) << 40)) return FA2_ERR_INVALID_ARG;
+  return FA2_OK;
 }
 
 fa2_status check_workspace(const void* ws, size_t bytes, size_t need) {
@@ -586,6 +610,31 @@ fa2_status fa2_fwd_varlen(const void* q, const void* k, const void* v, void* o, 
   return run_fwd(a, dtype, sq, sk, sv, so, static_cast<cudaStream_t>(stream));
 }
 
+fa2_status fa2_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                               int N, int H, int d, fa2_dtype dtype, fa2_strides sq, fa2_strides sk,
+                               fa2_strides sv, fa2_strides so, const uint8_t* block_mask,
+                               int64_t mask_stride_b, int64_t mask_stride_h, float softmax_scale,
+                               int causal, int window_left, int window_right,
+                               const float* alibi_slopes, float dropout_p,
+                               unsigned long long dropout_seed, void* stream) {
+  FA2_TRY(check_shape(B, N, H, d, dtype));
+  FA2_TRY(check_tensor(q, sq, dtype));
+  FA2_TRY(check_tensor(k, sk, dtype));
+  FA2_TRY(check_tensor(v, sv, dtype));
+  FA2_TRY(check_tensor(o, so, dtype));
+  if (lse == nullptr || !aligned16(lse)) return FA2_ERR_INVALID_ARG;
+  if (o == q || o == k || o == v) return FA2_ERR_INVALID_ARG;
+  FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
+  FA2_TRY(check_block_mask(block_mask, mask_stride_b, mask_stride_h));
+  AttnArgs a;
+  fill_fwd_args(&a, q, k, v, o, lse, B, N, H, d, sq, sk, sv, so, softmax_scale, causal, window_left,
+                window_right, alibi_slopes, dropout_p, dropout_seed);
+  a.block_mask = block_mask;
+  a.bm_sb = mask_stride_b;
+  a.bm_sh = mask_stride_h;
+  return run_fwd(a, dtype, sq, sk, sv, so, static_cast<cudaStream_t>(stream));
+}
+
 fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D, int B, int N, int H, int d,
                               fa2_dtype dtype, fa2_strides so, fa2_strides sdo, void* stream) {
   FA2_TRY(check_shape(B, N, H, d, dtype));
@@ -670,6 +719,36 @@ fa2_status fa2_bwd_varlen(const void* q, const void* k, const void* v, const voi
                 dropout_p, dropout_seed);
   a.cu_seqlens = cu_seqlens;
   a.total = total;
+  return run_bwd(a, dtype, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic,
+                 static_cast<cudaStream_t>(stream));
+}
+
+fa2_status fa2_bwd_blocksparse(const void* q, const void* k, const void* v, const void* dout,
+                               const float* lse, const float* D, void* dq, void* dk, void* dv,
+                               void* workspace, size_t workspace_bytes, int B, int N, int H, int d,
+                               fa2_dtype dtype, fa2_strides sq, fa2_strides sk, fa2_strides sv,
+                               fa2_strides sdo, fa2_strides sdq, fa2_strides sdk, fa2_strides sdv,
+                               const uint8_t* block_mask, int64_t mask_stride_b,
+                               int64_t mask_stride_h, float softmax_scale, int causal,
+                               int window_left, int window_right, const float* alibi_slopes,
+                               float dropout_p, unsigned long long dropout_seed, int deterministic,
+                               void* stream) {
+  FA2_TRY(check_shape(B, N, H, d, dtype));
+  for (auto [ptr, s] : {std::pair<const void*, fa2_strides>{q, sq}, {k, sk}, {v, sv}, {dout, sdo},
+                        {dq, sdq}, {dk, sdk}, {dv, sdv}})
+    FA2_TRY(check_tensor(ptr, s, dtype));
+  if (lse == nullptr || !aligned16(lse) || D == nullptr || !aligned16(D)) return FA2_ERR_INVALID_ARG;
+  FA2_TRY(check_options(softmax_scale, dropout_p, alibi_slopes));
+  FA2_TRY(check_block_mask(block_mask, mask_stride_b, mask_stride_h));
+  FA2_TRY(check_workspace(workspace, workspace_bytes,
+                          fa2_bwd_workspace_size(B, N, H, d, dtype, deterministic)));
+  AttnArgs a;
+  fill_bwd_args(&a, q, k, v, dout, lse, D, dq, dk, dv, workspace, B, N, H, d, sq, sk, sv, sdo, sdq,
+                sdk, sdv, softmax_scale, causal, window_left, window_right, alibi_slopes, dropout_p,
+                dropout_seed);
+  a.block_mask = block_mask;
+  a.bm_sb = mask_stride_b;
+  a.bm_sh = mask_stride_h;
   return run_bwd(a, dtype, sq, sk, sv, sdo, sdq, sdk, sdv, deterministic,
                  static_cast<cudaStream_t>(stream));
 }

@@ -79,7 +79,10 @@ struct FwdParams {
   float scale_log2;                    // softmax_scale * log2(e)
   unsigned long long wait_ns;          // bounded-wait limit
   DropoutParams drop;                  // used by the DROPOUT instantiations
-  unsigned int* sched;                 // packed: {next unit, finished CTAs}, 0 between calls
+  unsigned int* sched;                 // packed / block-sparse: {next unit, finished CTAs}, 0 between calls
+  const uint8_t* bmask;                // block-sparse: [B, H, nb, nb] 128 x 128 block mask
+  long long bm_sb, bm_sh;              // its batch and head strides (elements)
+  int nb;                              // ceil(N / 128): blocks per row and column of the mask
 };
 
 template <int HD>
@@ -122,14 +125,28 @@ __device__ __forceinline__ int unit_index(int k) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-// Unit index -> (head, sequence, its rows, first local query row, first KV
-// block, KV block count).  A unit whose query pair lies past the end of its
-// sequence (packed calls: shorter sequences) has nblk = 0.
+// Block-mask row of query block qb of head (b, h), or null past the last
+// query block.
+__device__ __forceinline__ const uint8_t* bm_row(const FwdParams& p, int b, int h, int qb) {
+  return qb < p.nb ? p.bmask + b * p.bm_sb + h * p.bm_sh + (long long)qb * p.nb : nullptr;
+}
+// Does either query tile of a unit (mask rows r0, r1) need key block kb?
+__device__ __forceinline__ bool pair_needs(const uint8_t* r0, const uint8_t* r1, int kb) {
+  return r0[kb] != 0 || (r1 != nullptr && r1[kb] != 0);
+}
+
+// Unit index -> (head, sequence, its rows, first local query row, first and
+// last KV block, KV block count).  A unit whose query pair lies past the end
+// of its sequence (packed calls: shorter sequences) has nblk = 0.  With a
+// block mask, the unit visits only the KV blocks either of its query tiles
+// needs (at least one: a unit whose rows see nothing still writes O = 0 and
+// LSE = -inf from one fully hidden block).
 struct Unit {
-  int h, b, bt, base, len, row0, blk_begin, nblk;
+  int h, b, bt, base, len, row0, first, last, nblk;
 };
-template <bool PACKED>
+template <int MODE>
 __device__ __forceinline__ Unit unit_of(const FwdParams& p, int L) {
+  constexpr bool PACKED = MODE == kLayoutPacked;
   Unit u;
   const int nhb = p.H * p.B;
   int pair, hb;
@@ -153,27 +170,59 @@ __device__ __forceinline__ Unit unit_of(const FwdParams& p, int L) {
     u.len = p.N;
   }
   u.row0 = pair * 256;
-  u.blk_begin = 0;
+  u.first = 0;
+  u.last = -1;
   u.nblk = 0;
   if (u.row0 < u.len) {
     const int row_end = min(u.len, u.row0 + 256);
     const int kv_lo = p.wl >= 0 ? max(0, u.row0 - p.wl) : 0;
     const int kv_hi = p.wr >= 0 ? min(u.len - 1, row_end - 1 + p.wr) : u.len - 1;
-    u.blk_begin = kv_lo / 128;
-    u.nblk = kv_hi / 128 - u.blk_begin + 1;
+    u.first = kv_lo / 128;
+    u.last = kv_hi / 128;
+    u.nblk = u.last - u.first + 1;
+    if (MODE == kLayoutSparse) {
+      const uint8_t* r0 = bm_row(p, u.b, u.h, 2 * pair);
+      const uint8_t* r1 = bm_row(p, u.b, u.h, 2 * pair + 1);
+      int cnt = 0, first = -1;
+      for (int kb = u.first; kb <= u.last; ++kb)
+        if (pair_needs(r0, r1, kb)) {
+          if (first < 0) first = kb;
+          ++cnt;
+        }
+      if (cnt > 0) {
+        u.first = first;
+        u.nblk = cnt;
+      } else {
+        u.nblk = 1;
+      }
+    }
   }
   return u;
 }
-// Packed calls: units differ in cost with the sequence lengths, which a
-// static schedule cannot see, so the CTAs take units from a shared counter in
-// longest-first order, each as it becomes free.  Returns the next non-empty
-// unit, or -1 when none is left.  Only the producer thread calls this.
-template <bool PACKED>
+
+// The KV block a unit visits after block kb.
+template <int MODE>
+__device__ __forceinline__ int next_block(const FwdParams& p, const Unit& u, int kb) {
+  if (MODE != kLayoutSparse) return kb + 1;
+  const int pair = u.row0 / 256;
+  const uint8_t* r0 = bm_row(p, u.b, u.h, 2 * pair);
+  const uint8_t* r1 = bm_row(p, u.b, u.h, 2 * pair + 1);
+  for (++kb; kb < u.last; ++kb)
+    if (pair_needs(r0, r1, kb)) break;
+  return kb;
+}
+
+// Packed and block-sparse calls: units differ in cost with the sequence
+// lengths or the block mask, which a static schedule cannot see, so the CTAs
+// take units from a shared counter, each as it becomes free.  Returns the
+// next non-empty unit, or -1 when none is left.  Only the producer thread
+// calls this.
+template <int MODE>
 __device__ __forceinline__ int fetch_unit(const FwdParams& p) {
   for (;;) {
     const int L = int(atomicAdd(p.sched, 1u));
     if (L >= p.num_units) return -1;
-    if (unit_of<PACKED>(p, L).nblk > 0) return L;
+    if (unit_of<MODE>(p, L).nblk > 0) return L;
   }
 }
 }  // namespace fwd_detail
@@ -190,9 +239,12 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-template <int HD, bool ALIBI, bool DROPOUT, bool PACKED>
+template <int HD, bool ALIBI, bool DROPOUT, int MODE>
 __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<HD>;
+  constexpr bool PACKED = MODE == kLayoutPacked;
+  constexpr bool SPARSE = MODE == kLayoutSparse;
+  constexpr bool DYN = PACKED || SPARSE;  // units taken from the shared counter
   constexpr int BM = C::BM, BN = C::BN, NQT = C::NQT, SLOTS = C::SLOTS;
   constexpr int NCH = HD / 64;  // 64-column (128-byte) boxes per tile row
   using namespace fwd_detail;
@@ -254,9 +306,9 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
     if (lane == 0) {
       int n = 0, k = 0, q_issued = 0;
       bool ok = true;
-      int L = PACKED ? fetch_unit<PACKED>(p) : unit_index(0);
+      int L = DYN ? fetch_unit<MODE>(p) : unit_index(0);
       for (;; ++k) {
-        if (PACKED) {  // hand the unit index (or the end mark -1) to the other roles
+        if (DYN) {  // hand the unit index (or the end mark -1) to the other roles
           const int r = k % C::RING;
           if (!wait_bar(ring_empty(r), ((k / C::RING) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + 3)) break;
           ring[r] = L;
@@ -265,8 +317,8 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
         } else if (L >= p.num_units) {
           break;
         }
-        const Unit u = unit_of<PACKED>(p, L);
-        const int L_next = PACKED ? fetch_unit<PACKED>(p) : unit_index(k + 1);
+        const Unit u = unit_of<MODE>(p, L);
+        const int L_next = DYN ? fetch_unit<MODE>(p) : unit_index(k + 1);
         const int qb = k & 1;
         if (!wait_bar(q_empty(qb), ((k >> 1) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + 2)) break;
         bar_arrive_expect_tx(q_full(qb), NQT * C::QT_BYTES);
@@ -275,8 +327,9 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
             tma_load_4d(smem_u32(sQ + (qb * NQT + t) * C::QT_BYTES + c * BM * 128), &p.tm_q, q_full(qb),
                         c * 64, u.h, u.base + u.row0 + t * BM, u.bt);
         q_issued = k + 1;
-        for (int it = 0; it < u.nblk && ok; ++it) {
-          const int kv0 = u.base + (u.blk_begin + it) * BN;
+        int kb = u.first;
+        for (int it = 0; it < u.nblk && ok; ++it, kb = next_block<MODE>(p, u, kb)) {
+          const int kv0 = u.base + (SPARSE ? kb : u.first + it) * BN;
           for (int which = 0; which < 2; ++which, ++n) {
             const int s = n % SLOTS;
             if (!wait_bar(slot_empty(s), ((n / SLOTS) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + which)) {
@@ -293,7 +346,7 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
         if (!ok) break;
         L = L_next;
       }
-      if (PACKED) {
+      if (DYN) {
         // The last CTA to finish taking units returns the counters to zero
         // for the next call that uses them.
         __threadfence();
@@ -334,7 +387,7 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
       bool ok = true;
       for (int k = 0; ok; ++k) {
         int L;
-        if (PACKED) {
+        if (DYN) {
           const int r = k % C::RING;
           ok = wait_bar(ring_full(r), (k / C::RING) & 1, ab, p.wait_ns, SITE_MMA + 8);
           if (!ok) break;
@@ -345,7 +398,7 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
           L = unit_index(k);
           if (L >= p.num_units) break;
         }
-        const Unit u = unit_of<PACKED>(p, L);
+        const Unit u = unit_of<MODE>(p, L);
         const int qb = k & 1;
         ok = wait_bar(q_full(qb), (k >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
         if (!ok) break;
@@ -420,7 +473,7 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
     bool ok = true;
     for (int k = 0; ok; ++k) {
       int L;
-      if (PACKED) {
+      if (DYN) {
         const int r = k % C::RING;
         ok = wait_bar(ring_full(r), (k / C::RING) & 1, ab, p.wait_ns, SITE_SOFT + 2);
         if (!__all_sync(0xffffffffu, ok)) break;
@@ -432,16 +485,22 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
         L = unit_index(k);
         if (L >= p.num_units) break;
       }
-      const Unit u = unit_of<PACKED>(p, L);
+      const Unit u = unit_of<MODE>(p, L);
       const int h = u.h, b = u.b;
+      // this tile's block-mask row (null: tile past the last query block)
+      const uint8_t* mrow = SPARSE ? bm_row(p, b, h, u.row0 / 128 + t) : nullptr;
       const int i = u.row0 + t * BM + r;  // local query row (>= len for padding rows)
       const int lo = p.wl >= 0 ? max(0, i - p.wl) : 0;
       const int hi = p.wr >= 0 ? min(u.len - 1, i + p.wr) : u.len - 1;
       float slope2 = 0.f;
       if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
       float m_run = -CUDART_INF_F, l_run = 0.f;
-      for (int it = 0; it < u.nblk; ++it) {
-        const int kv0 = (u.blk_begin + it) * BN;
+      int kb = u.first;
+      for (int it = 0; it < u.nblk; ++it, kb = next_block<MODE>(p, u, kb)) {
+        const int kv0 = (SPARSE ? kb : u.first + it) * BN;
+        // block hidden from this tile by the block mask (it is visited for
+        // the other tile of the pair, or to write a fully hidden unit)
+        const bool hidden = SPARSE && (mrow == nullptr || mrow[kb] == 0);
         ok = wait_bar(s_full(t), (g + it) & 1, ab, p.wait_ns, SITE_SOFT + 0);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -460,11 +519,11 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
 #pragma unroll
           for (int c = 0; c < BN; ++c) s[c] = fmaf(slope2, fabsf(fi - float(c)), s[c] * C2);
         }
-        if (!(kv0 >= lo && kv0 + BN - 1 <= hi)) {
+        if (hidden || !(kv0 >= lo && kv0 + BN - 1 <= hi)) {
 #pragma unroll
           for (int c = 0; c < BN; ++c) {
             const int j = kv0 + c;
-            if (j < lo || j > hi) s[c] = -CUDART_INF_F;
+            if (hidden || j < lo || j > hi) s[c] = -CUDART_INF_F;
           }
         }
         float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(const AttnArgs a) {
   const float slope = a.alibi ? a.alibi[h] : 0.f;
   float m = -CUDART_INF_F, l = 0.f;
   for (int j = lo; j <= hi; ++j) {
+    if (!block_kept(a, b, h, i, j)) continue;
     const T* kr = kb + j * a.sk.n;
     float part = 0.f;
 #pragma unroll
@@ -116,6 +117,7 @@ __global__ void __launch_bounds__(128) simt_bwd_dkdv_kernel(const AttnArgs a) {
   // queries i that see key j: lo(i) <= j <= hi(i)
   const int i_lo = queries_lo(a, j), i_hi = queries_hi(a, j, sv.len);
   for (int i = i_lo; i <= i_hi; ++i) {
+    if (!block_kept(a, b, h, i, j)) continue;
     const T* qr = qb + i * a.sq.n;
     const T* dor = dob + i * a.sdo.n;
     float qf[E], df[E], ps = 0.f, pd = 0.f;
@@ -178,6 +180,7 @@ __global__ void __launch_bounds__(128) simt_bwd_dq_kernel(const AttnArgs a) {
   const float slope = a.alibi ? a.alibi[h] : 0.f;
   const int lo = visible_lo(a, i), hi = visible_hi(a, i, sv.len);
   for (int j = lo; j <= hi; ++j) {
+    if (!block_kept(a, b, h, i, j)) continue;
     const T* kr = kb + j * a.sk.n;
     const T* vr = vb + j * a.sv.n;
     float kf[E], ps = 0.f, pd = 0.f;

@@ -37,7 +37,8 @@ NOALLOC_MAX_DQ_FLOATS = 4 * 1024 * 1024
 
 # Every symbol include/fa2.h declares.
 EXPORTED = ("fa2_fwd", "fa2_bwd_preprocess", "fa2_bwd_workspace_size", "fa2_bwd",
-            "fa2_fwd_varlen", "fa2_bwd_varlen", "fa2_strerror", "fa2_device_status",
+            "fa2_fwd_varlen", "fa2_bwd_varlen", "fa2_fwd_blocksparse", "fa2_bwd_blocksparse",
+            "fa2_strerror", "fa2_device_status",
             "fa2_set_wait_limit_ms", "fa2_kernel_launches", "fa2_bwd_noalloc")
 # Device status code of a packed call whose cu_seqlens was malformed.
 STATUS_BAD_SEQLENS = 0xF10
@@ -84,6 +85,14 @@ def load_library(path: str = LIB_PATH):
                                    i, i, i, i, i, i, s, s, s, s, s, s, s, f, i, i, i, vp, f, u64,
                                    i, vp]
     lib.fa2_bwd_varlen.restype = i
+    i64 = ctypes.c_int64
+    lib.fa2_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, s, s, s, s, vp, i64, i64,
+                                        f, i, i, i, vp, f, u64, vp]
+    lib.fa2_fwd_blocksparse.restype = i
+    lib.fa2_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                        i, i, i, i, i, s, s, s, s, s, s, s, vp, i64, i64, f, i, i, i,
+                                        vp, f, u64, i, vp]
+    lib.fa2_bwd_blocksparse.restype = i
     lib.fa2_strerror.argtypes = [i]
     lib.fa2_strerror.restype = ctypes.c_char_p
     lib.fa2_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), i]
@@ -136,6 +145,23 @@ def _seqlens(cu_seqlens: torch.Tensor) -> torch.Tensor:
     if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
         raise ValueError("cu_seqlens must be a 1-D int32 tensor of B + 1 offsets")
     return cu_seqlens.contiguous()
+
+
+BLOCK = 128  # side of a block-mask block
+
+
+def _block_mask(block_mask: torch.Tensor, B: int, H: int, N: int):
+    """(tensor, batch stride, head stride) of a [B, H, nb, nb] uint8 block mask
+    (batch and head strides may be 0: one mask shared)."""
+    nb = (N + BLOCK - 1) // BLOCK
+    if block_mask.dtype not in (torch.uint8, torch.bool) or block_mask.dim() != 4:
+        raise ValueError("block_mask must be a [B, H, nb, nb] uint8 or bool tensor")
+    if tuple(block_mask.shape) != (B, H, nb, nb):
+        raise ValueError(f"block_mask shape {tuple(block_mask.shape)} != {(B, H, nb, nb)}")
+    m = block_mask.view(torch.uint8) if block_mask.dtype == torch.bool else block_mask
+    if m.stride(3) != 1 or m.stride(2) != nb:
+        m = m.contiguous()
+    return m, m.stride(0), m.stride(1)
 
 
 def _ptr(t):
@@ -279,6 +305,55 @@ def bwd_varlen(dout, q, k, v, lse, D, cu_seqlens, max_seqlen, softmax_scale=None
     return dq, dk, dv
 
 
+def fwd_blocksparse(q, k, v, block_mask, softmax_scale=None, causal=False,
+                    window_size=(-1, -1), alibi_slopes=None, dropout_p=0.0, out=None, lse=None,
+                    stream=None, dropout_seed=0):
+    """Forward pass with a [B, H, ceil(N/128), ceil(N/128)] block mask (uint8
+    or bool; nonzero = the 128 x 128 block may be attended)."""
+    lib = load_library()
+    B, N, H, d = q.shape
+    m, msb, msh = _block_mask(block_mask, B, H, N)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    c, wl, wr = _window(causal, window_size)
+    st = lib.fa2_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, N, H, d,
+                                 _dtype_code(q), _strides(q), _strides(k), _strides(v),
+                                 _strides(out), _ptr(m), msb, msh, _scale(softmax_scale), c, wl,
+                                 wr, _ptr(alibi_slopes), float(dropout_p),
+                                 int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, _stream(stream))
+    _check(st, "fa2_fwd_blocksparse")
+    return out, lse
+
+
+def bwd_blocksparse(dout, q, k, v, lse, D, block_mask, softmax_scale=None, causal=False,
+                    window_size=(-1, -1), alibi_slopes=None, dropout_p=0.0, deterministic=False,
+                    dq=None, dk=None, dv=None, workspace=None, stream=None, dropout_seed=0):
+    """Backward pass with the forward's block mask; returns (dq, dk, dv)."""
+    lib = load_library()
+    B, N, H, d = q.shape
+    m, msb, msh = _block_mask(block_mask, B, H, N)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = workspace_size(B, N, H, d, q.dtype, deterministic)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    c, wl, wr = _window(causal, window_size)
+    st = lib.fa2_bwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(D),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), wbytes, B, N, H, d,
+                                 _dtype_code(q), _strides(q), _strides(k), _strides(v),
+                                 _strides(dout), _strides(dq), _strides(dk), _strides(dv),
+                                 _ptr(m), msb, msh, _scale(softmax_scale), c, wl, wr,
+                                 _ptr(alibi_slopes), float(dropout_p),
+                                 int(dropout_seed) & 0xFFFFFFFFFFFFFFFF, int(bool(deterministic)),
+                                 _stream(stream))
+    _check(st, "fa2_bwd_blocksparse")
+    return dq, dk, dv
+
+
 def device_status(clear=True) -> int:
     """Device status word (0 = no kernel gave up a bounded wait)."""
     code = ctypes.c_int(0)
@@ -358,3 +433,35 @@ def flash_attention_v2_varlen(q, k, v, cu_seqlens, max_seqlen, dropout_p=0.0,
     [total, H, d] and sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1."""
     return _Fa2VarlenFunction.apply(q, k, v, cu_seqlens, max_seqlen, dropout_p, softmax_scale,
                                     causal, window_size, alibi_slopes, deterministic)
+
+
+class _Fa2BlockSparseFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, block_mask, dropout_p, softmax_scale, causal, window_size,
+                alibi_slopes, deterministic):
+        seed = int(torch.randint(0, 2**63 - 1, (1,)).item()) if dropout_p > 0 else 0
+        out, lse = fwd_blocksparse(q, k, v, block_mask, softmax_scale, causal, window_size,
+                                   alibi_slopes, dropout_p, dropout_seed=seed)
+        ctx.save_for_backward(q, k, v, out, lse, block_mask, alibi_slopes)
+        ctx.opts = (dropout_p, softmax_scale, causal, window_size, deterministic, seed)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse, block_mask, alibi_slopes = ctx.saved_tensors
+        dropout_p, softmax_scale, causal, window_size, deterministic, seed = ctx.opts
+        dout = dout if dout.stride(-1) == 1 else dout.contiguous()
+        D = bwd_preprocess(out, dout)
+        dq, dk, dv = bwd_blocksparse(dout, q, k, v, lse, D, block_mask, softmax_scale, causal,
+                                     window_size, alibi_slopes, dropout_p, deterministic,
+                                     dropout_seed=seed)
+        return dq, dk, dv, None, None, None, None, None, None, None
+
+
+def flash_attention_v2_blocksparse(q, k, v, block_mask, dropout_p=0.0, softmax_scale=None,
+                                   causal=False, window_size=(-1, -1), alibi_slopes=None,
+                                   deterministic=False):
+    """Exact attention restricted to the 128 x 128 blocks a [B, H, nb, nb]
+    block mask keeps, with autograd support; q, k, v are [B, N, H, d]."""
+    return _Fa2BlockSparseFunction.apply(q, k, v, block_mask, dropout_p, softmax_scale, causal,
+                                         window_size, alibi_slopes, deterministic)

@@ -223,6 +223,46 @@ fa2_status fa2_bwd_varlen(const void* q, const void* k, const void* v, const voi
                           unsigned long long dropout_seed, int deterministic, void* stream);
 
 /*
+ * Block-sparse attention (named as future work in §6 of the "FlashAttention
+ * v2" article): the padded calls above with a 128 x 128 block mask.  Key j is
+ * hidden from query i unless byte
+ *     block_mask[b * mask_stride_b + h * mask_stride_h + (i / 128) * nb + j / 128]
+ * is nonzero, nb = ceil(N / 128), on top of the causal and window masks.
+ *
+ *   block_mask      DEVICE uint8 [B, H, nb, nb] (rows of nb bytes); owned by
+ *                   the caller; read, never written.
+ *   mask_stride_b, mask_stride_h
+ *                   its batch and head strides in bytes, >= 0; 0 shares one
+ *                   mask across the batch or across the heads.
+ *
+ * Every other argument means what it means for fa2_fwd / fa2_bwd (same
+ * layouts, workspace size, dropout counter).  Blocks the mask hides are
+ * neither loaded nor multiplied.  A query row that sees no key gets O = 0,
+ * LSE = -inf and zero gradients.  The mask must be the same for the forward
+ * and the backward call.
+ */
+fa2_status fa2_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int N, int H, int d, fa2_dtype dtype,
+                               fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides so,
+                               const uint8_t* block_mask, int64_t mask_stride_b,
+                               int64_t mask_stride_h,
+                               float softmax_scale, int causal, int window_left,
+                               int window_right, const float* alibi_slopes, float dropout_p,
+                               unsigned long long dropout_seed, void* stream);
+
+fa2_status fa2_bwd_blocksparse(const void* q, const void* k, const void* v, const void* dout,
+                               const float* lse, const float* D, void* dq, void* dk, void* dv,
+                               void* workspace, size_t workspace_bytes,
+                               int B, int N, int H, int d, fa2_dtype dtype,
+                               fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides sdo,
+                               fa2_strides sdq, fa2_strides sdk, fa2_strides sdv,
+                               const uint8_t* block_mask, int64_t mask_stride_b,
+                               int64_t mask_stride_h,
+                               float softmax_scale, int causal, int window_left,
+                               int window_right, const float* alibi_slopes, float dropout_p,
+                               unsigned long long dropout_seed, int deterministic, void* stream);
+
+/*
  * fa2_bwd_noalloc: the bf16 backward pass without any caller-provided or
  * library-allocated workspace.  (No counterpart in the paper: this is an
  * interface convenience, not part of the method.)

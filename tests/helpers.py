@@ -76,7 +76,8 @@ def check_fwd(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what="", o_max=None):
     return float(err.max()), float(lerr.max())
 
 
-def d_rounding_bounds(q, k, do, o, scale, causal=False, wl=-1, wr=-1, slope=None):
+def d_rounding_bounds(q, k, do, o, scale, causal=False, wl=-1, wr=-1, slope=None,
+                      block_mask=None):
     """Per-element bounds on the error a bf16 dQ and dK carry because
     D = rowsum(dO o O) is formed from the bf16-rounded O (the backward pass
     takes O as an input), for one head.
@@ -91,7 +92,7 @@ def d_rounding_bounds(q, k, do, o, scale, causal=False, wl=-1, wr=-1, slope=None
     is no longer exact in bf16.  P comes from the oracle's scores and O is
     the oracle's output."""
     q, k, do, o = (np.asarray(x, dtype=np.float64) for x in (q, k, do, o))
-    s = oa.head_scores(q, k, np.arange(q.shape[0]), scale, causal, wl, wr, slope)
+    s = oa.head_scores(q, k, np.arange(q.shape[0]), scale, causal, wl, wr, slope, block_mask)
     m = s.max(axis=1, keepdims=True)
     p = np.exp(s - np.where(np.isfinite(m), m, 0.0))
     p /= np.maximum(p.sum(axis=1, keepdims=True), 1e-300)

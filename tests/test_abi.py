@@ -150,3 +150,24 @@ def test_bwd_varlen_checks_its_workspace(lib):
     args[11] = None                     # no cu_seqlens
     args[10] = need
     assert lib.fa2_bwd_varlen(*args) == F.FA2_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------- block-sparse
+def call_fwd_bs(lib, **kw):
+    a = dict(q=P, k=P, v=P, o=ctypes.c_void_p(0x200000), lse=P, mask=ctypes.c_void_p(0x800000),
+             sb=0, sh=0, d=128, dropout=0.0)
+    a.update(kw)
+    return lib.fa2_fwd_blocksparse(a["q"], a["k"], a["v"], a["o"], a["lse"], 1, 256, 2, a["d"],
+                                   F.FA2_BF16, S128, S128, S128, S128, a["mask"], a["sb"], a["sh"],
+                                   0.0, 0, -1, -1, None, a["dropout"], 0, None)
+
+
+@pytest.mark.parametrize("bad", [dict(mask=None), dict(sb=-1), dict(sh=-4), dict(d=80),
+                                 dict(q=None), dict(o=P), dict(dropout=2.0)])
+def test_fwd_blocksparse_rejects_invalid(lib, bad):
+    assert call_fwd_bs(lib, **bad) == F.FA2_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_valid_blocksparse_call_without_device_is_cuda_error(lib):
+    assert call_fwd_bs(lib) == F.FA2_ERR_CUDA
