@@ -394,6 +394,7 @@ def run_gpu(args):
         line["dropout"] = run_dropout(F, W)
         line["packed"] = run_packed(F, W)
         line["blocksparse"] = run_blocksparse(F, W)
+        line["fp8"] = run_fp8(F, W)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -529,6 +530,29 @@ def run_blocksparse(F, W):
             "blocks": nb * nb, "fwd_ms": round(tf, 4),
             "fwd_tflops": round(ff / (tf * 1e-3) / 1e12, 1), "bwd_ms": round(tb, 4),
             "bwd_tflops": round(2.5 * ff / (tb * 1e-3) / 1e12, 1)}
+
+
+def run_fp8(F, W):
+    """e4m3 forward of the bench workload (B=8 H=16 N=2048 d=128), causal and
+    not, against the e4m3 dense peak taken as twice the measured bf16 burst
+    peak (the nominal e4m3 : bf16 ratio of the tensor cores)."""
+    import torch
+    peaks, src = load_peaks()
+    fp8_peak = 2.0 * float(peaks["bf16_tflops"])
+    res = []
+    for causal in (False, True):
+        w = W.mid(causal)
+        q8, k8, v8, (qd, kd, vd) = W.make_fp8_inputs(w, "cuda")
+        out, lse = F.fwd_fp8(q8, k8, v8, qd, kd, vd, causal=causal)
+        tf, _ = _time_pair(lambda: F.fwd_fp8(q8, k8, v8, qd, kd, vd, causal=causal, out=out, lse=lse),
+                           lambda: None)
+        tfl = flops_fwd(w.B, w.H, w.N, w.d, causal) / (tf * 1e-3) / 1e12
+        res.append({"workload": "B=8 H=16 N=2048 d=128 e4m3", "causal": causal,
+                    "fwd_ms": round(tf, 4), "fwd_tflops": round(tfl, 1),
+                    "frac_of_e4m3_peak": round(tfl / fp8_peak, 3),
+                    "e4m3_peak": f"2 x {src} bf16_tflops = {fp8_peak:.0f}"})
+        del q8, k8, v8, out, lse
+    return res
 
 
 def run_sweep(F, W, args, full=False):

@@ -54,6 +54,8 @@ struct AttnArgs {
   int wl, wr;         // window bounds, negative = unbounded
   int dropout;        // nonzero: apply the dropout mask described in philox.cuh
   DropoutParams drop;
+  float descale_qk;   // e4m3 inputs: q_descale * k_descale (else 1)
+  float descale_v;    // e4m3 inputs: v_descale (else 1)
 };
 
 // One sequence of a call: batch coordinate `bt` and first row `row0` of its

@@ -153,6 +153,22 @@ fa2_status encode_bf16_4d(CUtensorMap* m, const void* ptr, const fa2_strides& s,
   return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
 }
 
+// The same map over an e4m3 [B, N, H, d] tensor (bytes): box (128, 1, 128,
+// 1), one 128-byte swizzled row per tile row at d = 128.
+fa2_status encode_u8_4d(CUtensorMap* m, const void* ptr, const fa2_strides& s, int B, int N, int H,
+                        int d) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  FA2_TRY(get_encoder(&enc));
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(s.h), cuuint64_t(s.n), cuuint64_t(s.b)};
+  cuuint32_t box[4] = {128, 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
+}
+
 // 3-D map over the fp32 dQ accumulator [B*H, N, d] (dense): dims (d, N, B*H),
 // box (32, 32, 1) -- one warp's 32 rows -- 128-byte swizzle; used for TMA
 // bulk reductions.
@@ -231,16 +247,22 @@ fa2_status dispatch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa
                               const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
                               int causal_order, cudaStream_t st);
 
-template <int HD, bool ALIBI, bool DROPOUT, int MODE>
+template <int HD, bool ALIBI, bool DROPOUT, int MODE, bool FP8 = false>
 fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_strides& sk,
                             const fa2_strides& sv, const fa2_strides& so, int dev, int sm_count,
                             int causal_order, cudaStream_t st) {
   static std::atomic<uint64_t> mask{0};
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
-  FA2_TRY(encode_input(&p.tm_q, a.q, sq, a, HD));
-  FA2_TRY(encode_input(&p.tm_k, a.k, sk, a, HD));
-  FA2_TRY(encode_input(&p.tm_v, a.v, sv, a, HD));
+  if (FP8) {
+    FA2_TRY(encode_u8_4d(&p.tm_q, a.q, sq, a.B, a.N, a.H, HD));
+    FA2_TRY(encode_u8_4d(&p.tm_k, a.k, sk, a.B, a.N, a.H, HD));
+    FA2_TRY(encode_u8_4d(&p.tm_v, a.v, sv, a.B, a.N, a.H, HD));
+  } else {
+    FA2_TRY(encode_input(&p.tm_q, a.q, sq, a, HD));
+    FA2_TRY(encode_input(&p.tm_k, a.k, sk, a, HD));
+    FA2_TRY(encode_input(&p.tm_v, a.v, sv, a, HD));
+  }
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.so_b = a.cu_seqlens ? 0 : so.b;
   p.so_n = so.n;
@@ -258,7 +280,8 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.npairs = (a.N + 255) / 256;
   p.num_units = p.npairs * a.H * a.B;
   p.heavy_first = causal_order;
-  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.scale_log2 = a.scale * a.descale_qk * 1.4426950408889634f;
+  p.o_scale = a.descale_v;
   p.wait_ns = g_wait_ns.load();
   p.drop = a.drop;
   p.bmask = a.block_mask;
@@ -266,12 +289,12 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.bm_sh = a.bm_sh;
   p.nb = (a.N + 127) / 128;
   if (MODE != kLayoutPadded) FA2_TRY(sched_counters(dev, &p.sched));
-  auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, MODE>;
-  constexpr int smem = FwdCfg<HD>::SMEM_BYTES;
+  auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, MODE, FP8>;
+  constexpr int smem = FwdCfg<HD, FP8>::SMEM_BYTES;
   FA2_TRY(ensure_smem(kern, smem, dev, mask));
   // persistent grid: one CTA per SM (shared memory and TMEM allow one)
   const unsigned grid = unsigned(std::min(p.num_units, std::max(sm_count, 1)));
-  kern<<<grid, FwdCfg<HD>::THREADS, smem, st>>>(p);
+  kern<<<grid, FwdCfg<HD, FP8>::THREADS, smem, st>>>(p);
   return launched(1);
 }
 
@@ -453,6 +476,8 @@ void fill_common(AttnArgs* a, int B, int N, int H, int d, float softmax_scale, i
   normalise_window(causal, &a->wl, &a->wr);
   a->dropout = dropout_p != 0.f;
   a->drop = make_dropout(dropout_p, dropout_seed);
+  a->descale_qk = 1.f;
+  a->descale_v = 1.f;
 }
 
 void fill_fwd_args(AttnArgs* a, const void* q, const void* k, const void* v, void* o, float* lse,
@@ -633,6 +658,42 @@ fa2_status fa2_fwd_blocksparse(const void* q, const void* k, const void* v, void
   a.bm_sb = mask_stride_b;
   a.bm_sh = mask_stride_h;
   return run_fwd(a, dtype, sq, sk, sv, so, static_cast<cudaStream_t>(stream));
+}
+
+fa2_status fa2_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N,
+                       int H, int d, fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides so,
+                       float q_descale, float k_descale, float v_descale, float softmax_scale,
+                       int causal, int window_left, int window_right, const float* alibi_slopes,
+                       void* stream) {
+  FA2_TRY(check_shape(B, N, H, d, FA2_BF16));
+  // e4m3 tensors: strides in bytes must keep rows 16-byte aligned (the
+  // check for a 1-byte type is the fp32 one with four times the stride)
+  for (auto [ptr, s] : {std::pair<const void*, fa2_strides>{q, sq}, {k, sk}, {v, sv}}) {
+    if (s.b % 16 != 0 || s.n % 16 != 0 || s.h % 16 != 0) return FA2_ERR_INVALID_ARG;
+    FA2_TRY(check_tensor(ptr, s, FA2_BF16));
+  }
+  FA2_TRY(check_tensor(o, so, FA2_BF16));
+  if (lse == nullptr || !aligned16(lse)) return FA2_ERR_INVALID_ARG;
+  if (o == q || o == k || o == v) return FA2_ERR_INVALID_ARG;
+  FA2_TRY(check_options(softmax_scale, 0.f, alibi_slopes));
+  for (float x : {q_descale, k_descale, v_descale})
+    if (!(x > 0.f) || std::isinf(x)) return FA2_ERR_INVALID_ARG;
+  if (d != 128) return FA2_ERR_UNSUPPORTED;
+  AttnArgs a;
+  fill_fwd_args(&a, q, k, v, o, lse, B, N, H, d, sq, sk, sv, so, softmax_scale, causal, window_left,
+                window_right, alibi_slopes, 0.f, 0);
+  a.descale_qk = q_descale * k_descale;
+  a.descale_v = v_descale;
+  int dev;
+  DeviceInfo di;
+  FA2_TRY(current_device(&dev, &di));
+  if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;
+  const int heavy_first = (a.wr >= 0 || a.wl >= 0) ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return a.alibi ? launch_fwd_sm100<128, true, false, kLayoutPadded, true>(a, sq, sk, sv, so, dev,
+                                                                          di.sm_count, heavy_first, st)
+                 : launch_fwd_sm100<128, false, false, kLayoutPadded, true>(a, sq, sk, sv, so, dev,
+                                                                           di.sm_count, heavy_first, st);
 }
 
 fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D, int B, int N, int H, int d,

@@ -79,21 +79,24 @@ struct FwdParams {
   float scale_log2;                    // softmax_scale * log2(e)
   unsigned long long wait_ns;          // bounded-wait limit
   DropoutParams drop;                  // used by the DROPOUT instantiations
+  float o_scale;                       // e4m3 inputs: V's dequantisation factor (else 1)
   unsigned int* sched;                 // packed / block-sparse: {next unit, finished CTAs}, 0 between calls
   const uint8_t* bmask;                // block-sparse: [B, H, nb, nb] 128 x 128 block mask
   long long bm_sb, bm_sh;              // its batch and head strides (elements)
   int nb;                              // ceil(N / 128): blocks per row and column of the mask
 };
 
-template <int HD>
+template <int HD, bool FP8 = false>
 struct FwdCfg {
   static constexpr int BM = 128;        // query rows per tile
   static constexpr int BN = 128;        // keys per KV block
   static constexpr int NQT = 2;         // query tiles per unit
   static constexpr int QBUFS = 2;       // Q double buffer (across units)
-  static constexpr int SLOTS = HD == 128 ? 3 : 8;
-  static constexpr int QT_BYTES = BM * HD * 2;
-  static constexpr int KV_BYTES = BN * HD * 2;
+  static constexpr int ESZ = FP8 ? 1 : 2;                    // bytes per element
+  static constexpr int KSTEP = FP8 ? 32 : 16;                // K of one MMA
+  static constexpr int SLOTS = FP8 ? 6 : (HD == 128 ? 3 : 8);
+  static constexpr int QT_BYTES = BM * HD * ESZ;
+  static constexpr int KV_BYTES = BN * HD * ESZ;
   static constexpr int OFF_KV = QBUFS * NQT * QT_BYTES;
   static constexpr int OFF_BARS = OFF_KV + SLOTS * KV_BYTES;
   static constexpr int RING = 4;        // unit-index ring of the packed scheduler
@@ -239,14 +242,17 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-template <int HD, bool ALIBI, bool DROPOUT, int MODE>
+template <int HD, bool ALIBI, bool DROPOUT, int MODE, bool FP8 = false>
 __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<HD>;
+  using C = FwdCfg<HD, FP8>;
+  static_assert(!FP8 || (HD == 128 && !DROPOUT && MODE == kLayoutPadded),
+                "e4m3 inputs: d = 128, padded layout, no dropout");
   constexpr bool PACKED = MODE == kLayoutPacked;
   constexpr bool SPARSE = MODE == kLayoutSparse;
   constexpr bool DYN = PACKED || SPARSE;  // units taken from the shared counter
   constexpr int BM = C::BM, BN = C::BN, NQT = C::NQT, SLOTS = C::SLOTS;
-  constexpr int NCH = HD / 64;  // 64-column (128-byte) boxes per tile row
+  constexpr int NCH = HD * C::ESZ / 128;  // 128-byte boxes per tile row
+  constexpr int KSTEP = C::KSTEP;
   using namespace fwd_detail;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
         for (int t = 0; t < NQT; ++t)
           for (int c = 0; c < NCH; ++c)
             tma_load_4d(smem_u32(sQ + (qb * NQT + t) * C::QT_BYTES + c * BM * 128), &p.tm_q, q_full(qb),
-                        c * 64, u.h, u.base + u.row0 + t * BM, u.bt);
+                        c * (128 / C::ESZ), u.h, u.base + u.row0 + t * BM, u.bt);
         q_issued = k + 1;
         int kb = u.first;
         for (int it = 0; it < u.nblk && ok; ++it, kb = next_block<MODE>(p, u, kb)) {
@@ -339,8 +345,8 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
             bar_arrive_expect_tx(slot_full(s), C::KV_BYTES);
             const CUtensorMap* tm = which == 0 ? &p.tm_k : &p.tm_v;
             for (int c = 0; c < NCH; ++c)
-              tma_load_4d(smem_u32(sKV + s * C::KV_BYTES + c * BN * 128), tm, slot_full(s), c * 64, u.h, kv0,
-                          u.bt);
+              tma_load_4d(smem_u32(sKV + s * C::KV_BYTES + c * BN * 128), tm, slot_full(s),
+                          c * (128 / C::ESZ), u.h, kv0, u.bt);
           }
         }
         if (!ok) break;
@@ -364,24 +370,36 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t id_qk = idesc_bf16_f32(BM, BN, 0, 0);
-      const uint32_t id_pv = idesc_bf16_f32(BM, HD, 0, 1);
+      const uint32_t id_qk = FP8 ? idesc_e4m3_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
+      const uint32_t id_pv = FP8 ? idesc_e4m3_f32(BM, HD, 0, 1) : idesc_bf16_f32(BM, HD, 0, 1);
+      // One MMA covers KSTEP elements of K = 32 bytes of a 128-byte swizzled
+      // row; four of them fill a row, then the next 128-byte box follows.
       auto qk = [&](int t, int qb, int s) {
         const uint32_t a0 = smem_u32(sQ + (qb * NQT + t) * C::QT_BYTES), b0 = smem_u32(sKV + s * C::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
+        for (int kk = 0; kk < HD / KSTEP; ++kk) {
           const uint32_t ao = (kk / 4) * (BM * 128) + (kk % 4) * 32;
           const uint32_t bo = (kk / 4) * (BN * 128) + (kk % 4) * 32;
-          umma_ss(tmem + t * 128, sdesc_sw128(a0 + ao, 16, 1024), sdesc_sw128(b0 + bo, 16, 1024),
-                  id_qk, kk > 0);
+          if (FP8)
+            umma_ss_f8(tmem + t * 128, sdesc_sw128(a0 + ao, 16, 1024), sdesc_sw128(b0 + bo, 16, 1024),
+                       id_qk, kk > 0);
+          else
+            umma_ss(tmem + t * 128, sdesc_sw128(a0 + ao, 16, 1024), sdesc_sw128(b0 + bo, 16, 1024),
+                    id_qk, kk > 0);
         }
       };
+      // P from TMEM (KSTEP keys = 8 columns per MMA), V MN-major: KSTEP key
+      // rows of 128 bytes per MMA, 128-byte column chunks BN * 128 apart.
       auto pv = [&](int t, int s, bool acc) {
         const uint32_t v0 = smem_u32(sKV + s * C::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(tmem + 256 + t * HD, tmem + t * 128 + kk * 8,
-                  sdesc_sw128(v0 + kk * 2048, BN * 128, 1024), id_pv, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / KSTEP; ++kk) {
+          const uint64_t vd = sdesc_sw128(v0 + kk * KSTEP * 128, BN * 128, 1024);
+          if (FP8)
+            umma_ts_f8(tmem + 256 + t * HD, tmem + t * 128 + kk * 8, vd, id_pv, (acc || kk > 0) ? 1u : 0u);
+          else
+            umma_ts(tmem + 256 + t * HD, tmem + t * 128 + kk * 8, vd, id_pv, (acc || kk > 0) ? 1u : 0u);
+        }
       };
       int n = 0, g = 0;  // KV slots, blocks
       bool ok = true;
@@ -568,8 +586,20 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
         // one generator call per quad of rows and 16 keys (the rows of a quad
         // share i / 4: row0 is a multiple of 256), applied as 16-bit masks to
         // the packed pairs.
+        if (FP8) {
+          // e4m3 P: four per column, 32 columns.  P <= 2^TAU = 256 < 448.
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
+          for (int c = 0; c < BN / 64; ++c) {
+            uint32_t w16[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              w16[e] = pack_e4m3x4(s[c * 64 + 4 * e], s[c * 64 + 4 * e + 1], s[c * 64 + 4 * e + 2],
+                                   s[c * 64 + 4 * e + 3]);
+            tmem_st16(s_addr + c * 16, w16);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < (FP8 ? 0 : BN / 32); ++c) {
           uint32_t w16[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) w16[e] = pack_bf16(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]);
@@ -611,7 +641,7 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = l_run > 0.f ? (DROPOUT ? p.drop.keep_scale : 1.f) / l_run : 0.f;
+      const float inv_l = l_run > 0.f ? (DROPOUT ? p.drop.keep_scale : (FP8 ? p.o_scale : 1.f)) / l_run : 0.f;
       // the sequence's rows, looked up again here rather than kept live
       // through the block loop
       const SeqView sv = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};

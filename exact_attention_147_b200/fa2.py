@@ -38,6 +38,7 @@ NOALLOC_MAX_DQ_FLOATS = 4 * 1024 * 1024
 # Every symbol include/fa2.h declares.
 EXPORTED = ("fa2_fwd", "fa2_bwd_preprocess", "fa2_bwd_workspace_size", "fa2_bwd",
             "fa2_fwd_varlen", "fa2_bwd_varlen", "fa2_fwd_blocksparse", "fa2_bwd_blocksparse",
+            "fa2_fwd_fp8",
             "fa2_strerror", "fa2_device_status",
             "fa2_set_wait_limit_ms", "fa2_kernel_launches", "fa2_bwd_noalloc")
 # Device status code of a packed call whose cu_seqlens was malformed.
@@ -93,6 +94,9 @@ def load_library(path: str = LIB_PATH):
                                         i, i, i, i, i, s, s, s, s, s, s, s, vp, i64, i64, f, i, i, i,
                                         vp, f, u64, i, vp]
     lib.fa2_bwd_blocksparse.restype = i
+    lib.fa2_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, s, s, s, s, f, f, f, f, i, i, i, vp,
+                                vp]
+    lib.fa2_fwd_fp8.restype = i
     lib.fa2_strerror.argtypes = [i]
     lib.fa2_strerror.restype = ctypes.c_char_p
     lib.fa2_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), i]
@@ -352,6 +356,28 @@ def bwd_blocksparse(dout, q, k, v, lse, D, block_mask, softmax_scale=None, causa
                                  _stream(stream))
     _check(st, "fa2_bwd_blocksparse")
     return dq, dk, dv
+
+
+def fwd_fp8(q, k, v, q_descale, k_descale, v_descale, softmax_scale=None, causal=False,
+            window_size=(-1, -1), alibi_slopes=None, out=None, lse=None, stream=None):
+    """Forward pass on e4m3 inputs (torch.float8_e4m3fn, [B, N, H, 128]) with
+    per-tensor dequantisation factors; returns (out bf16, lse fp32)."""
+    lib = load_library()
+    for t in (q, k, v):
+        if t.dtype != torch.float8_e4m3fn:
+            raise TypeError("fwd_fp8 takes torch.float8_e4m3fn tensors")
+    B, N, H, d = q.shape
+    if out is None:
+        out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    c, wl, wr = _window(causal, window_size)
+    st = lib.fa2_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, N, H, d, _strides(q),
+                         _strides(k), _strides(v), _strides(out), float(q_descale),
+                         float(k_descale), float(v_descale), _scale(softmax_scale), c, wl, wr,
+                         _ptr(alibi_slopes), _stream(stream))
+    _check(st, "fa2_fwd_fp8")
+    return out, lse
 
 
 def device_status(clear=True) -> int:

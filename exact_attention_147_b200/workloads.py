@@ -99,6 +99,26 @@ def make_inputs(w: Workload, device: str | torch.device = "cpu",
     return tuple(out)
 
 
+def make_fp8_inputs(w: Workload, device: str | torch.device = "cpu"):
+    """e4m3 inputs for workload ``w``: q, k, v drawn as in make_inputs (fp32,
+    before any cast), each divided by its descale factor max|x| / 448 so that
+    it spans the e4m3 range, then cast to torch.float8_e4m3fn.  Returns
+    (q8, k8, v8, (q_descale, k_descale, v_descale)); the dequantised inputs
+    are x8 * descale."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    shape = (w.B, w.N, w.H, w.d)
+    out, scales = [], []
+    for std in (w.q_std, w.k_std, w.v_std):
+        t = torch.randn(shape, generator=g, dtype=torch.float32)
+        if std != 1.0:
+            t.mul_(std)
+        ds = float(t.abs().max()) / 448.0
+        out.append((t / ds).to(torch.float8_e4m3fn).to(device))
+        scales.append(ds)
+    return out[0], out[1], out[2], tuple(scales)
+
+
 # ---------------------------------------------------------------------------
 # The five workload families.
 # ---------------------------------------------------------------------------

@@ -263,6 +263,34 @@ fa2_status fa2_bwd_blocksparse(const void* q, const void* k, const void* v, cons
                                unsigned long long dropout_seed, int deterministic, void* stream);
 
 /*
+ * FP8 forward (the FlashAttention-3 page lists FP8 support as a further
+ * speed-up; it gives no numerics, so this is the plain reading): q, k and v
+ * are e4m3 (float8 e4m3fn: 1 sign, 4 exponent, 3 mantissa bits, max 448)
+ * with per-tensor dequantisation factors, and the result is the attention of
+ * the dequantised values q_descale * q, k_descale * k, v_descale * v.
+ *
+ *   q, k, v        [B, N, H, d] e4m3 bytes; strides in elements (= bytes),
+ *                  multiples of 16; base pointers 16-byte aligned.
+ *   o              [B, N, H, d] bf16 output, strides multiples of 8.
+ *   lse            [B, H, N] fp32, as for fa2_fwd.
+ *   q_descale, k_descale, v_descale
+ *                  finite, > 0.
+ *   d              128 only (FA2_ERR_UNSUPPORTED otherwise).
+ *
+ * Both products run on the tensor cores in e4m3 with fp32 accumulation: the
+ * scores exactly (products of e4m3 values are exact in fp32), and P V with
+ * the probabilities rounded to e4m3 (relative error <= 2^-4, or 2^-10
+ * absolute below the normal range; the softmax statistics and LSE stay
+ * fp32).  No dropout; the masks and ALiBi work as for fa2_fwd.
+ */
+fa2_status fa2_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int N, int H, int d,
+                       fa2_strides sq, fa2_strides sk, fa2_strides sv, fa2_strides so,
+                       float q_descale, float k_descale, float v_descale,
+                       float softmax_scale, int causal, int window_left, int window_right,
+                       const float* alibi_slopes, void* stream);
+
+/*
  * fa2_bwd_noalloc: the bf16 backward pass without any caller-provided or
  * library-allocated workspace.  (No counterpart in the paper: this is an
  * interface convenience, not part of the method.)

@@ -120,3 +120,25 @@ def check_grad(g_gpu, g_ref, dtype, what="", floor=0.0):
     assert not over.any(), (f"{what}: grad max err {err:.3e} > bound "
                             f"{np.max(bound):.3e} at {np.argwhere(over)[0]} (max|ref| {scale:.3e})")
     return float(err), float(scale)
+
+
+def fp8_o_bound(q, k, v, scale, causal=False, wl=-1, wr=-1, slope=None):
+    """Per-element bound on the O error of the e4m3 forward, for one head
+    (q, k, v: the dequantised inputs in float64).
+
+    The scores are exact (e4m3 products are exact in fp32).  P enters the
+    PV product rounded to e4m3 as p = P_ij * c with P_ij = exp(s_ij - m_i)
+    <= 1 and c >= 1 (the kernel's running max never exceeds the row max);
+    the rounding error of p is at most max(2^-4 p, 2^-10) (3 mantissa bits;
+    half the subnormal spacing), and dividing by l * c leaves at most
+    sum_j max(2^-4 P_ij, 2^-10 [P_ij > 0]) |v_jc| / l_i, l_i = sum_j P_ij.
+    O is then rounded to bf16: 2^-8 |O|.  A 1e-6 relative term covers the
+    fp32 accumulation."""
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    s = oa.head_scores(q, k, np.arange(q.shape[0]), scale, causal, wl, wr, slope)
+    m = s.max(axis=1, keepdims=True)
+    P = np.exp(s - np.where(np.isfinite(m), m, 0.0))
+    l = np.maximum(P.sum(axis=1, keepdims=True), 1e-300)
+    err_p = np.where(P > 0, np.maximum(2.0 ** -4 * P, 2.0 ** -10), 0.0)
+    o = (P @ v) / l
+    return (err_p @ np.abs(v)) / l + 2.0 ** -8 * np.abs(o) + 1e-6 * (P @ np.abs(v)) / l

@@ -171,3 +171,26 @@ def test_fwd_blocksparse_rejects_invalid(lib, bad):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
 def test_valid_blocksparse_call_without_device_is_cuda_error(lib):
     assert call_fwd_bs(lib) == F.FA2_ERR_CUDA
+
+
+# ----------------------------------------------------------------- e4m3 forward
+S8 = F.Strides(2048 * 16 * 128, 16 * 128, 128)   # e4m3 [B, N, H=16, 128] (bytes)
+
+
+def call_fwd_fp8(lib, **kw):
+    a = dict(q=P, o=ctypes.c_void_p(0x200000), d=128, sq=S8, qd=1.0)
+    a.update(kw)
+    return lib.fa2_fwd_fp8(a["q"], P, P, a["o"], P, 1, 256, 16, a["d"], a["sq"], S8, S8, S128,
+                           a["qd"], 1.0, 1.0, 0.0, 0, -1, -1, None, None)
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(o=P), dict(qd=0.0), dict(qd=float("inf")),
+                                 dict(qd=float("nan")), dict(sq=F.Strides(8, 16 * 128, 128)),
+                                 dict(d=100)])
+def test_fwd_fp8_rejects_invalid(lib, bad):
+    assert call_fwd_fp8(lib, **bad) == F.FA2_ERR_INVALID_ARG
+
+
+def test_fwd_fp8_head_dim_64_unsupported(lib):
+    assert call_fwd_fp8(lib, d=64, sq=F.Strides(2048 * 16 * 64, 16 * 64, 64)) == \
+        F.FA2_ERR_UNSUPPORTED
