@@ -143,35 +143,21 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ dist
 def dist_setup(n_gpus):
-    import torch
+    """One process per GPU over NCCL (see exact_attention_147_b200.ranks)."""
+    from exact_attention_147_b200 import ranks
     if n_gpus <= 1 and "WORLD_SIZE" not in os.environ:
         return 0, 1, 0
-    import datetime
-
-    import torch.distributed as dist
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                            device_id=torch.device("cuda", local))
-    return rank, world, local
+    return ranks.init("nccl", timeout_s=120.0)
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    from exact_attention_147_b200 import ranks
+    ranks.barrier(world)
 
 
 def max_over_ranks(x, world):
-    if world <= 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from exact_attention_147_b200 import ranks
+    return ranks.max_over_ranks(x, world, "cuda")
 
 
 # ------------------------------------------------------------------ oracle arm
@@ -259,7 +245,8 @@ def run_gpu(args):
     F.load_library()
     w = dict(WORKLOAD)
     B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
-    wl = W.Workload("bench", B=B, N=N, H=H, d=d, causal=causal, seed=1000 + rank)
+    from exact_attention_147_b200 import ranks
+    wl = W.Workload("bench", B=B, N=N, H=H, d=d, causal=causal, seed=ranks.batch_seed(1000, rank))
     q, k, v, do = W.make_inputs(wl, "cuda")
     out = torch.empty_like(q)
     lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
@@ -313,7 +300,7 @@ def run_gpu(args):
     f_fwd = flops_fwd(B, H, N, d, causal)
     f_step = 3.5 * f_fwd
     ms_step = ms_total / args.steps
-    value = world * f_step / (ms_step * 1e-3) / 1e12
+    value = ranks.whole_job_rate(f_step, world, ms_step * 1e-3) / 1e12
 
     # ---- end to end: pinned host buffers, copies inside the timed region
     e2e = None
@@ -344,7 +331,7 @@ def run_gpu(args):
         ms_e2e = max_over_ranks(s2.elapsed_time(t2), world) / args.steps
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
         d2h = sum(t.numel() * t.element_size() for t in houts) + hlse.numel() * 4
-        e2e = {"value": world * f_step / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": ranks.whole_job_rate(f_step, world, ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
 
     peaks, peak_src = load_peaks()
@@ -397,9 +384,7 @@ def run_gpu(args):
         line["fp8"] = run_fp8(F, W)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    ranks.finalize(world)
     return 0
 
 
