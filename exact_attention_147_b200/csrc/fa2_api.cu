@@ -292,6 +292,14 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, MODE, FP8>;
   constexpr int smem = FwdCfg<HD, FP8>::SMEM_BYTES;
   FA2_TRY(ensure_smem(kern, smem, dev, mask));
+  // The kernel re-balances registers between its warpgroups; the shares add
+  // up to 512 threads x REGS_AT_LAUNCH, so it must launch with that many per
+  // thread, or a warpgroup's increase would wait forever.
+  {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return FA2_ERR_CUDA;
+    if (fa.numRegs < FwdCfg<HD, FP8>::REGS_AT_LAUNCH) return FA2_ERR_UNSUPPORTED;
+  }
   // persistent grid: one CTA per SM (shared memory and TMEM allow one)
   const unsigned grid = unsigned(std::min(p.num_units, std::max(sm_count, 1)));
   kern<<<grid, FwdCfg<HD, FP8>::THREADS, smem, st>>>(p);

@@ -101,12 +101,19 @@ struct FwdCfg {
   static constexpr int OFF_BARS = OFF_KV + SLOTS * KV_BYTES;
   static constexpr int RING = 4;        // unit-index ring of the packed scheduler
   // q_full[2], q_empty[2], slot full/empty, s_full[2], p_ready[2], o_full[2],
-  // o_empty[2], drain, ring full[4], ring empty[4]
-  static constexpr int NBARS = 2 * QBUFS + 2 * SLOTS + 4 * NQT + 1 + 2 * RING;
-  // barriers, then the TMEM address, the abort flag, 2 spare words and the ring
-  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16 + 4 * RING;
+  // o_empty[2], drain, ring full[4], ring empty[4], stats_full[2], stats_free[2]
+  static constexpr int NBARS = 2 * QBUFS + 2 * SLOTS + 4 * NQT + 1 + 2 * RING + 2 * NQT;
+  // barriers, then the TMEM address, the abort flag, 2 spare words, the ring
+  // and the per-row results (1 / l, LSE) the softmax hands to the epilogue
+  static constexpr int OFF_STATS = OFF_BARS + NBARS * 8 + 16 + 4 * RING;
+  static constexpr int SMEM_BYTES = OFF_STATS + NQT * BM * 8;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 512;
+  // registers per thread after re-balancing (launch: 128 x 512 = 65536):
+  // softmax warpgroups 184, epilogue warpgroup 80, loader / MMA warpgroup 64
+  static constexpr int REGS_SOFT = HD == 128 ? 184 : 176, REGS_EPI = 80, REGS_MISC = HD == 128 ? 64 : 80;
+  static constexpr int REGS_AT_LAUNCH = (2 * 128 * REGS_SOFT + 128 * REGS_EPI + 128 * REGS_MISC) / 512;
+  static_assert(REGS_AT_LAUNCH == 128, "register split must use exactly the launch budget");
 };
 
 namespace fwd_detail {
@@ -243,7 +250,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 }
 
 template <int HD, bool ALIBI, bool DROPOUT, int MODE, bool FP8 = false>
-__global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<HD, FP8>;
   static_assert(!FP8 || (HD == 128 && !DROPOUT && MODE == kLayoutPadded),
                 "e4m3 inputs: d = 128, padded layout, no dropout");
@@ -275,9 +282,12 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
   const uint32_t drain_bar = bar0 + 8u * (12 + 2 * SLOTS);
   auto ring_full = [&](int r) { return bar0 + 8u * (13 + 2 * SLOTS + r); };
   auto ring_empty = [&](int r) { return bar0 + 8u * (13 + 2 * SLOTS + C::RING + r); };
+  auto stats_full = [&](int t) { return bar0 + 8u * (13 + 2 * SLOTS + 2 * C::RING + t); };
+  auto stats_free = [&](int t) { return bar0 + 8u * (15 + 2 * SLOTS + 2 * C::RING + t); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* ring = abort_flag + 3;  // packed: unit indices handed from the producer to the other roles
+  float2* stats = reinterpret_cast<float2*>(smem_raw + C::OFF_STATS);  // [NQT][BM] (1 / l, LSE)
   AbortFlag ab{abort_flag};
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -288,16 +298,19 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
       const uint32_t bar = bar0 + 8u * i;
       uint32_t cnt = 1;
       if (bar == p_ready(0) || bar == p_ready(1) || bar == o_empty(0) || bar == o_empty(1)) cnt = 128;
-      if (bar >= ring_empty(0) && bar <= ring_empty(C::RING - 1)) cnt = 9;  // MMA + 8 softmax warps
+      if (bar == stats_full(0) || bar == stats_full(1) || bar == stats_free(0) || bar == stats_free(1))
+        cnt = 128;
+      // MMA + 8 softmax warps + 4 epilogue warps
+      if (bar >= ring_empty(0) && bar <= ring_empty(C::RING - 1)) cnt = 13;
       bar_init(bar, cnt);
     }
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
@@ -307,7 +320,9 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp >= 12) {
+    regs_dec<C::REGS_MISC>();
+  if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int n = 0, k = 0, q_issued = 0;
@@ -367,7 +382,7 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
       for (int j = (n > SLOTS ? n - SLOTS : 0); j < n; ++j)
         drain_wait(slot_full(j % SLOTS), (j / SLOTS) & 1, p.wait_ns);
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = FP8 ? idesc_e4m3_f32(BM, BN, 0, 0) : idesc_bf16_f32(BM, BN, 0, 0);
@@ -479,7 +494,73 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
       umma_commit(drain_bar);
       drain_wait(drain_bar, 0, p.wait_ns);
     }
+  }
+  } else if (warp >= 8) {
+    regs_dec<C::REGS_EPI>();
+    // ------------------------------------------------------------ epilogue
+    // One thread per TMEM lane (query row) of both tiles: takes the row's
+    // 1 / l and LSE from the softmax, reads O_t out of TMEM as soon as its
+    // last PV product has landed, releases the TMEM columns and stores the
+    // normalised row, while the softmax warps already work on the next unit.
+    const int r = (warp % 4) * 32 + lane;
+    const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
+    const float o_mult = DROPOUT ? p.drop.keep_scale : (FP8 ? p.o_scale : 1.f);
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      int L;
+      if (DYN) {
+        const int rr = k % C::RING;
+        ok = wait_bar(ring_full(rr), (k / C::RING) & 1, ab, p.wait_ns, SITE_SOFT + 3);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        L = ring[rr];
+        __syncwarp();
+        if (lane == 0) bar_arrive(ring_empty(rr));
+        if (L < 0) break;
+      } else {
+        L = unit_index(k);
+        if (L >= p.num_units) break;
+      }
+      const Unit u = unit_of<MODE>(p, L);
+      const SeqView sv = PACKED ? seq_view(p.cu_seqlens, u.b, p.N, p.total) : SeqView{u.b, 0, p.N};
+      for (int t = 0; t < NQT && ok; ++t) {
+        const int i = u.row0 + t * BM + r;  // local query row (>= len for padding rows)
+        ok = wait_bar(stats_full(t), k & 1, ab, p.wait_ns, SITE_SOFT + 4);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const float2 st = stats[t * BM + r];  // (1 / l, LSE)
+        bar_arrive(stats_free(t));
+        ok = wait_bar(o_full(t), k & 1, ab, p.wait_ns, SITE_SOFT + 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float inv_l = st.x * o_mult;
+        const uint32_t o_addr = tmem + lane_base + 256 + t * HD;
+        __nv_bfloat16* orow = p.o + sv.bt * p.so_b + (long long)(sv.row0 + i) * p.so_n + u.h * p.so_h;
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t w32[32];
+          tmem_ld32(o_addr + c * 32, w32);
+          tmem_ld_wait();
+          if (c == HD / 32 - 1) {  // O_t has been read: the next unit may overwrite it
+            tc_fence_before();
+            bar_arrive(o_empty(t));
+          }
+          uint32_t w16[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w16[e] = pack_bf16(__uint_as_float(w32[2 * e]) * inv_l, __uint_as_float(w32[2 * e + 1]) * inv_l);
+          if (i < sv.len) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) =
+                  make_uint4(w16[4 * q4], w16[4 * q4 + 1], w16[4 * q4 + 2], w16[4 * q4 + 3]);
+          }
+        }
+        if (i < sv.len) p.lse[(size_t(sv.bt) * p.H + u.h) * (PACKED ? p.stat_rows : p.N) + sv.row0 + i] = st.y;
+      }
+    }
   } else {
+    regs_inc<C::REGS_SOFT>();
     // ------------------------------------------------------------ softmax
     const int t = warp / 4;
     const int r = (warp % 4) * 32 + lane;
@@ -636,46 +717,22 @@ __global__ void __launch_bounds__(320, 1) fa2_fwd_sm100_kernel(const __grid_cons
         bar_arrive(p_ready(t));
       }
       if (!ok) break;
-      // -------------------------------------------------------- epilogue
-      ok = wait_bar(o_full(t), k & 1, ab, p.wait_ns, SITE_SOFT + 1);
+      // ------------------------------------ hand the row's results over
+      // (the epilogue warps normalise and store O; this buffer is reused
+      // once they have read it)
+      ok = wait_bar(stats_free(t), (k & 1) ^ 1, ab, p.wait_ns, SITE_SOFT + 5);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      tc_fence_after();
-      const float inv_l = l_run > 0.f ? (DROPOUT ? p.drop.keep_scale : (FP8 ? p.o_scale : 1.f)) / l_run : 0.f;
-      // the sequence's rows, looked up again here rather than kept live
-      // through the block loop
-      const SeqView sv = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};
-      __nv_bfloat16* orow = p.o + sv.bt * p.so_b + (long long)(sv.row0 + i) * p.so_n + h * p.so_h;
-#pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t w32[32];
-        tmem_ld32(o_addr + c * 32, w32);
-        tmem_ld_wait();
-        if (c == HD / 32 - 1) {  // O_t has been read: the next unit may overwrite it
-          tc_fence_before();
-          bar_arrive(o_empty(t));
-        }
-        uint32_t w16[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w16[e] = pack_bf16(__uint_as_float(w32[2 * e]) * inv_l, __uint_as_float(w32[2 * e + 1]) * inv_l);
-        if (i < sv.len) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) =
-                make_uint4(w16[4 * q4], w16[4 * q4 + 1], w16[4 * q4 + 2], w16[4 * q4 + 3]);
-        }
-      }
-      if (i < sv.len)
-        p.lse[(size_t(sv.bt) * p.H + h) * (PACKED ? p.stat_rows : p.N) + sv.row0 + i] =
-            l_run > 0.f ? (m_run + log2f(l_run)) * LN2 : -CUDART_INF_F;
+      stats[t * BM + r] = make_float2(l_run > 0.f ? 1.f / l_run : 0.f,
+                                      l_run > 0.f ? (m_run + log2f(l_run)) * LN2 : -CUDART_INF_F);
+      bar_arrive(stats_full(t));
       g += u.nblk;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
