@@ -315,8 +315,9 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         float* side = sSide + sq * 256;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          side[lane + 32 * e] = l2v[e];
-          side[128 + lane + 32 * e] = dvv[e];
+          // stored negated: the compute warps add them with paired FMAs
+          side[lane + 32 * e] = -l2v[e];
+          side[128 + lane + 32 * e] = -dvv[e];
         }
         __threadfence_block();
         __syncwarp();
@@ -468,18 +469,18 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const int c = h2 * 32 + e;
-          const float4 l4 = *reinterpret_cast<const float4*>(side + c);
+          const float4 l4 = *reinterpret_cast<const float4*>(side + c);  // -LSE log2(e)
           float x0, x1, x2, x3;
           if (ALIBI) {
-            x0 = fmaf(slope2, fabsf(fj + float(c)), fmaf(__uint_as_float(u[e]), C2, -l4.x));
-            x1 = fmaf(slope2, fabsf(fj + float(c + 1)), fmaf(__uint_as_float(u[e + 1]), C2, -l4.y));
-            x2 = fmaf(slope2, fabsf(fj + float(c + 2)), fmaf(__uint_as_float(u[e + 2]), C2, -l4.z));
-            x3 = fmaf(slope2, fabsf(fj + float(c + 3)), fmaf(__uint_as_float(u[e + 3]), C2, -l4.w));
+            x0 = fmaf(slope2, fabsf(fj + float(c)), fmaf(__uint_as_float(u[e]), C2, l4.x));
+            x1 = fmaf(slope2, fabsf(fj + float(c + 1)), fmaf(__uint_as_float(u[e + 1]), C2, l4.y));
+            x2 = fmaf(slope2, fabsf(fj + float(c + 2)), fmaf(__uint_as_float(u[e + 2]), C2, l4.z));
+            x3 = fmaf(slope2, fabsf(fj + float(c + 3)), fmaf(__uint_as_float(u[e + 3]), C2, l4.w));
           } else {
-            x0 = fmaf(__uint_as_float(u[e]), C2, -l4.x);
-            x1 = fmaf(__uint_as_float(u[e + 1]), C2, -l4.y);
-            x2 = fmaf(__uint_as_float(u[e + 2]), C2, -l4.z);
-            x3 = fmaf(__uint_as_float(u[e + 3]), C2, -l4.w);
+            const uint64_t c2x2 = pk2(C2, C2);
+            upk2(fma2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), c2x2, pk2(l4.x, l4.y)), x0, x1);
+            upk2(fma2(pk2(__uint_as_float(u[e + 2]), __uint_as_float(u[e + 3])), c2x2, pk2(l4.z, l4.w)), x2,
+                 x3);
           }
           pr[c] = ex2(x0);
           pr[c + 1] = ex2(x1);
@@ -552,7 +553,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
           const int cc = c * 32 + 2 * e;
-          const float4 d4 = *reinterpret_cast<const float4*>(side + 128 + cc);
+          const float4 d4 = *reinterpret_cast<const float4*>(side + 128 + cc);  // -D
           float g0 = __uint_as_float(u[2 * e]), g1 = __uint_as_float(u[2 * e + 1]);
           float g2 = __uint_as_float(u[2 * e + 2]), g3 = __uint_as_float(u[2 * e + 3]);
           if (DROPOUT) {  // dP = (dO V^T) o keep / (1 - p)
@@ -561,8 +562,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
             g2 = kept(cc + 2) ? g2 * p.drop.keep_scale : 0.f;
             g3 = kept(cc + 3) ? g3 * p.drop.keep_scale : 0.f;
           }
-          w[e] = pack_bf16(pr[cc] * (g0 - d4.x), pr[cc + 1] * (g1 - d4.y));
-          w[e + 1] = pack_bf16(pr[cc + 2] * (g2 - d4.z), pr[cc + 3] * (g3 - d4.w));
+          float s0, s1, s2, s3;  // dS = P o (dP - D), two at a time
+          upk2(mul2(pk2(pr[cc], pr[cc + 1]), add2(pk2(g0, g1), pk2(d4.x, d4.y))), s0, s1);
+          upk2(mul2(pk2(pr[cc + 2], pr[cc + 3]), add2(pk2(g2, g3), pk2(d4.z, d4.w))), s2, s3);
+          w[e] = pack_bf16(s0, s1);
+          w[e + 1] = pack_bf16(s2, s3);
         }
         // written over columns this thread has already read
         tmem_st16(tmem + lane_base + T_DP + cq + c * 16, w);

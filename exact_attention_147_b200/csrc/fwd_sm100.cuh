@@ -625,13 +625,15 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             if (hidden || j < lo || j > hi) s[c] = -CUDART_INF_F;
           }
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        // Row maximum: four independent chains of three-input maxima.
+        float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]);
+        float mx2 = fmaxf(s[4], s[5]), mx3 = fmaxf(s[6], s[7]);
 #pragma unroll
-        for (int c = 4; c < BN; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
+        for (int c = 8; c < BN; c += 8) {
+          mx0 = max3(mx0, s[c], s[c + 1]);
+          mx1 = max3(mx1, s[c + 2], s[c + 3]);
+          mx2 = max3(mx2, s[c + 4], s[c + 5]);
+          mx3 = max3(mx3, s[c + 6], s[c + 7]);
         }
         float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
         if (!ALIBI) mx *= C2;  // now in base-2 units
@@ -642,26 +644,23 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
           m_run = mx;
         }
         const float m_use = m_run == -CUDART_INF_F ? 0.f : m_run;
-        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+        // Exponentials, with the scale-and-shift and the row sum done on
+        // pairs of scores (one paired instruction for two).
+        const uint64_t c2x2 = pk2(ALIBI ? 1.f : C2, ALIBI ? 1.f : C2);
+        const uint64_t negm2 = pk2(-m_use, -m_use);
+        uint64_t l2x[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < BN; c += 4) {
-          if (ALIBI) {
-            s[c] = ex2(s[c] - m_use);
-            s[c + 1] = ex2(s[c + 1] - m_use);
-            s[c + 2] = ex2(s[c + 2] - m_use);
-            s[c + 3] = ex2(s[c + 3] - m_use);
-          } else {
-            s[c] = ex2(fmaf(s[c], C2, -m_use));
-            s[c + 1] = ex2(fmaf(s[c + 1], C2, -m_use));
-            s[c + 2] = ex2(fmaf(s[c + 2], C2, -m_use));
-            s[c + 3] = ex2(fmaf(s[c + 3], C2, -m_use));
-          }
-          l0 += s[c];
-          l1 += s[c + 1];
-          l2 += s[c + 2];
-          l3 += s[c + 3];
+        for (int c = 0; c < BN; c += 2) {
+          float x0, x1;
+          upk2(fma2(pk2(s[c], s[c + 1]), c2x2, negm2), x0, x1);
+          s[c] = ex2(x0);
+          s[c + 1] = ex2(x1);
+          l2x[(c / 2) % 4] = add2(l2x[(c / 2) % 4], pk2(s[c], s[c + 1]));
         }
-        l_run = fmaf(l_run, alpha, (l0 + l1) + (l2 + l3));
+        float la, lb, lc, ld;
+        upk2(add2(l2x[0], l2x[1]), la, lb);
+        upk2(add2(l2x[2], l2x[3]), lc, ld);
+        l_run = fmaf(l_run, alpha, (la + lb) + (lc + ld));
         // P (bf16 pairs) over the first BN/2 columns of S.  With dropout, l
         // keeps the un-dropped sum and dropped probabilities leave P here:
         // one generator call per quad of rows and 16 keys (the rows of a quad
