@@ -68,6 +68,8 @@ struct BwdParams {
   float scale_log2;                      // c * log2(e)
   unsigned long long wait_ns;
   DropoutParams drop;                    // used by the DROPOUT instantiations
+  int num_items;                         // key blocks x heads x batch (kernel 1 work items)
+  unsigned int* sched;                   // packed / block-sparse kernel 1: {next item, finished CTAs}
 };
 
 template <int HD>
@@ -86,16 +88,18 @@ struct BwdCfg {
   static constexpr int OFF_STG = OFF_SIDE + Q_STAGES * SIDE_BYTES;  // dQ staging ring
   static constexpr int STG_BYTES = 2 * 16384;                         // 2 x (128 rows x 32 fp32)
   static constexpr int OFF_BARS = OFF_STG + STG_BYTES;
+  static constexpr int RING = 4;                      // item-index ring (packed / block-sparse)
   // kv_full, Q full/empty, dO full/empty, s_full, dp_full, p_ready, ds_ready,
-  // dq_full, dq_free, acc_full, drain
-  static constexpr int NBARS = 1 + 2 * Q_STAGES + 2 * DO_STAGES + 8;
+  // dq_full, dq_free, acc_full, drain, kv_empty, acc_empty, ring full/empty
+  static constexpr int NBARS = 1 + 2 * Q_STAGES + 2 * DO_STAGES + 8 + 2 + 2 * RING;
   // No alignment slack: the kernel checks that the dynamic shared memory
   // starts on a 1024-byte boundary (it does: the reserved 1 KB precedes it).
-  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16;
+  // barriers, then the TMEM address, the abort flag, 2 spare words, the ring
+  static constexpr int SMEM_BYTES = OFF_BARS + NBARS * 8 + 16 + 4 * RING;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static constexpr int THREADS = 512;
   // registers per thread after the warpgroup re-balancing (see kernel 1)
-  static constexpr int REGS_COMPUTE = 144, REGS_DRAIN = 160, REGS_MISC = 64;
+  static constexpr int REGS_COMPUTE = 136, REGS_DRAIN = 136, REGS_MISC = 104;
   static constexpr int REGS_AT_LAUNCH = (2 * 128 * REGS_COMPUTE + 128 * REGS_DRAIN + 128 * REGS_MISC) / 512;
   static_assert(REGS_AT_LAUNCH == 128, "register split must use exactly the launch budget");
 };
@@ -162,10 +166,86 @@ __device__ __forceinline__ int count_kept(const uint8_t* m, long long stride, in
   return cnt;
 }
 
+// One work item of kernel 1: a 128-key block of one (batch, head), and the
+// query blocks it visits ([qb_first, qb_last], only the kept ones with a
+// block mask; nq of them).  An item past the end of a shorter packed
+// sequence is empty.
+struct BItem {
+  int h, b, kb, k0, len, bt, trow, qb_first, qb_last, nq;
+  const uint8_t* mcol;  // block-sparse: this key block's mask column (mcol[qb * nb])
+  size_t head_off;      // row statistics of local row 0
+  bool empty;
+};
+
+template <int MODE>
+__device__ __forceinline__ BItem item_of(const BwdParams& p, int I) {
+  BItem it;
+  const int nhb = p.H * p.B;
+  int hb;
+  if (p.heavy_first) {  // masks: key block 0 of every head first (it sees the most queries)
+    it.kb = I / nhb;
+    hb = I % nhb;
+  } else {              // key blocks of one head together (they share its Q and dO in L2)
+    it.kb = I % p.nblocks;
+    hb = I / p.nblocks;
+  }
+  it.h = hb % p.H;
+  it.b = hb / p.H;
+  const SeqView sv = MODE == kLayoutPacked ? seq_view(p.cu_seqlens, it.b, p.N, p.total)
+                                           : SeqView{it.b, 0, p.N};
+  it.len = sv.len;
+  it.bt = sv.bt;
+  it.trow = sv.row0;
+  it.k0 = it.kb * 128;
+  it.empty = it.k0 >= it.len;
+  it.mcol = nullptr;
+  it.qb_first = 0;
+  it.qb_last = -1;
+  it.nq = 0;
+  it.head_off = (size_t(sv.bt) * p.H + it.h) * (MODE == kLayoutPacked ? p.stat_rows : p.N) + sv.row0;
+  if (!it.empty) {
+    const int k_last = min(it.len - 1, it.k0 + 127);
+    const int i_lo = p.wr >= 0 ? max(0, it.k0 - p.wr) : 0;
+    const int i_hi = p.wl >= 0 ? min(it.len - 1, k_last + p.wl) : it.len - 1;
+    it.qb_first = i_lo / 128;
+    it.qb_last = i_hi / 128;
+    if (MODE == kLayoutSparse) {
+      it.mcol = p.bmask + it.b * p.bm_sb + it.h * p.bm_sh + it.kb;
+      it.nq = count_kept(it.mcol, p.nb, it.qb_first, it.qb_last);
+    } else {
+      it.nq = it.qb_last - it.qb_first + 1;
+    }
+  }
+  return it;
+}
+
+// The query block a work item visits after block qb.
+template <int MODE>
+__device__ __forceinline__ int next_qblock(const BwdParams& p, const BItem& it, int qb) {
+  return MODE == kLayoutSparse ? next_kept(it.mcol, p.nb, qb, it.qb_last) : qb + 1;
+}
+
+// Static schedule of kernel 1 (padded calls): the k-th item of CTA c in a
+// persistent grid of G CTAs, a snake over the item order.
+__device__ __forceinline__ int bwd_item_index(int k) {
+  const int G = int(gridDim.x), c = int(blockIdx.x);
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
+}
+
+// Packed / block-sparse calls: items taken from a shared counter as CTAs
+// become free (their cost follows the lengths or the mask).  Next non-empty
+// item, or -1.  Only the producer thread calls this.
+template <int MODE>
+__device__ __forceinline__ int fetch_item(const BwdParams& p) {
+  for (;;) {
+    const int I = int(atomicAdd(p.sched, 1u));
+    if (I >= p.num_items) return -1;
+    if (!item_of<MODE>(p, I).empty) return I;
+  }
+}
+
 // Writes the same 16 words straight to row `row` of a global bf16 tensor
-// (columns col0 .. col0 + 31): the output path of tiles whose last rows
-// belong to the next sequence of a packed batch, which a TMA store of the
-// whole tile would overwrite.
+// (columns col0 .. col0 + 31).
 __device__ __forceinline__ void st_global_row32(__nv_bfloat16* base, const Strides& s, const SeqView& v,
                                                 int row, int h, int col0, const uint32_t (&w)[16]) {
   __nv_bfloat16* dst = row_ptr<__nv_bfloat16>(base, s, v, row, h) + col0;
@@ -178,24 +258,37 @@ __device__ __forceinline__ void st_global_row32(__nv_bfloat16* base, const Strid
 // ---------------------------------------------------------------------------
 // Kernel 1: dK, dV (and the atomically accumulated dQ when WITH_DQ)
 //
+// Persistent: one CTA per SM walks work items (a 128-key block of one head),
+// so barriers, TMEM and registers are set up once and one item's tail
+// overlaps the next one's start: the MMA warp releases K and V as soon as
+// the item's last products have read them and the loader brings the next
+// item's K and V while the compute warps write dK and dV out of TMEM.
+//
 // 16 warps: warpgroups 0 and 1 compute (thread = key row; warpgroup w owns
 // query columns [64w, 64w+64) of every S^T / dP^T tile), warpgroup 2 drains
 // dQ (thread = query row), warp 12 loads, warp 13 issues the MMAs.  Register
-// budget after the split: compute 144, drain 160, loader/MMA warpgroup 64
-// (2*128*144 + 128*160 + 128*64 = 65536 = 512 threads x 128 at launch; the
-// host checks the launch register count before every launch).
+// budget after the split: compute 136, drain 136, loader/MMA warpgroup 104
+// (the loader and the MMA warp follow their own item schedule) (2*128*136 +
+// 128*136 + 128*104 = 65536 = 512 threads x 128 at launch; the host checks
+// the launch register count before every launch).
 //
 // dQ path: the drain warpgroup reads the whole dQ tile out of TMEM into
 // registers, releases the TMEM columns (the next dP^T reuses them), then
 // stages it 32 columns at a time through a two-slot shared-memory ring and
 // adds it into the fp32 accumulator with TMA bulk reductions, which go
 // through the TMA unit rather than the load/store queues.
+//
+// Barrier phases run on two counters kept identically by every role: jn,
+// the items this CTA has processed (kv_full / kv_empty / acc_full /
+// acc_empty), and g, the query blocks it has processed (the Q / dO rings
+// and the per-block barriers).
 // ---------------------------------------------------------------------------
 template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT, int MODE>
 __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<HD>;
   constexpr bool PACKED = MODE == kLayoutPacked;
   constexpr bool SPARSE = MODE == kLayoutSparse;
+  constexpr bool DYN = PACKED || SPARSE;  // items taken from the shared counter
   using namespace bwd_detail;
   constexpr int QS = C::Q_STAGES, DS = C::DO_STAGES;
   constexpr int NCH = HD / 64;
@@ -224,47 +317,27 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   const uint32_t s_full = b0 + 8u * (1 + 2 * QS + 2 * DS);
   const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24;
   const uint32_t dq_full = s_full + 32, dq_free = s_full + 40, acc_full = s_full + 48;
-  const uint32_t drain_bar = b0 + 8u * (C::NBARS - 1);
+  const uint32_t drain_bar = s_full + 56;
+  const uint32_t kv_empty = s_full + 64, acc_empty = s_full + 72;
+  auto ring_full = [&](int r) { return s_full + 80 + 8u * r; };
+  auto ring_empty = [&](int r) { return s_full + 80 + 8u * (C::RING + r); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* ring = abort_flag + 3;  // item indices handed from the loader to the other roles
   AbortFlag ab{abort_flag};
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int wg = warp / 4;
-  const int nhb = p.H * p.B;
-  int kb, hb;
-  if (p.heavy_first) {  // causal: key block 0 is seen by the most query blocks
-    kb = int(blockIdx.x / nhb);
-    hb = int(blockIdx.x % nhb);
-  } else {
-    kb = int(blockIdx.x % p.nblocks);
-    hb = int(blockIdx.x / p.nblocks);
-  }
-  const int h = hb % p.H, b = hb / p.H;
-  const SeqView sv = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};
-  const int len = sv.len;
-  const int k0 = kb * 128;        // local key row of this block
-  if (k0 >= len) return;          // past the end of a shorter packed sequence: no work
-  const int k_last = min(len - 1, k0 + 127);
-  const int i_lo = p.wr >= 0 ? max(0, k0 - p.wr) : 0;
-  const int i_hi = p.wl >= 0 ? min(len - 1, k_last + p.wl) : len - 1;
-  // query blocks visited: [qb_first, qb_last], only the kept ones when a
-  // block mask is given (this key block's mask column: mcol[qb * nb])
-  int qb_first = i_lo / 128;
-  const int qb_last = i_hi / 128;
-  const uint8_t* mcol = SPARSE ? p.bmask + b * p.bm_sb + h * p.bm_sh + kb : nullptr;
-  const int nq = SPARSE ? count_kept(mcol, p.nb, qb_first, qb_last) : qb_last - qb_first + 1;
-  auto next_qb = [&](int qb) { return SPARSE ? next_kept(mcol, p.nb, qb, qb_last) : qb + 1; };
-  const size_t head_off = (size_t(sv.bt) * p.H + h) * (PACKED ? p.stat_rows : p.N) + sv.row0;
-  const int trow = sv.row0;       // tensor row of local row 0
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int i = 0; i < C::NBARS; ++i) {
       const uint32_t bar = b0 + 8u * i;
       uint32_t cnt = 1;
-      if (bar == p_ready || bar == ds_ready) cnt = 256;
+      if (bar == p_ready || bar == ds_ready || bar == acc_empty) cnt = 256;
       if (bar == dq_free) cnt = 128;
+      // MMA thread + 8 compute warps + 4 drain warps
+      if (bar >= ring_empty(0) && bar <= ring_empty(C::RING - 1)) cnt = 13;
       bar_init(bar, cnt);
     }
     fence_barrier_init();
@@ -278,76 +351,147 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // The next item of a consumer role (MMA, compute, drain): the ring entry
+  // the loader published (DYN), or the static schedule; -1 at the end.
+  // `k` counts the schedule entries this role has looked at.  Returns false
+  // when a wait gave up.
+  auto next_item = [&](int& k, int& I, bool warp_wide, int site) -> bool {
+    for (;;) {
+      if (DYN) {
+        const int rr = k % C::RING;
+        bool ok = wait_bar(ring_full(rr), (k / C::RING) & 1, ab, p.wait_ns, site);
+        if (warp_wide) ok = __all_sync(0xffffffffu, ok);
+        if (!ok) return false;
+        I = ring[rr];
+        if (warp_wide) __syncwarp();
+        if (!warp_wide || lane == 0) bar_arrive(ring_empty(rr));
+        ++k;
+        return true;  // the loader publishes only non-empty items, then -1
+      }
+      I = bwd_item_index(k++);
+      if (I >= p.num_items) {
+        I = -1;
+        return true;
+      }
+      if (!item_of<MODE>(p, I).empty) return true;
+    }
+  };
+
   if (wg == 3) {
     regs_dec<C::REGS_MISC>();
     if (warp == 12) {
       // ---------------------------------------------------------- producer
-      if (lane == 0) {
-        bar_arrive_expect_tx(kv_full, 2 * C::TILE);
-        for (int c = 0; c < NCH; ++c) {
-          tma_load_4d(smem_u32(sK + c * 16384), &p.tm_k, kv_full, c * 64, h, trow + k0, sv.bt);
-          tma_load_4d(smem_u32(sV + c * 16384), &p.tm_v, kv_full, c * 64, h, trow + k0, sv.bt);
-        }
-      }
-      int issued_q = 0, issued_do = 0;
+      int issued_q = 0, issued_do = 0, issued_kv = 0, jn = 0, g = 0, k = 0;
       bool ok = true;
-      int qb = qb_first;
-      for (int it = 0; it < nq && ok; ++it, qb = next_qb(qb)) {
-        const int i0 = (SPARSE ? qb : qb_first + it) * 128;
-        const int sq = it % QS;
-        // log2-scaled LSE and D of this query block, +inf / 0 past the end; loaded
-        // before waiting for the slot so the latency overlaps the wait
-        float l2v[4], dvv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = i0 + lane + 32 * e;
-          l2v[e] = CUDART_INF_F;
-          dvv[e] = 0.f;
-          if (i < len) {
-            const float l = p.lse[head_off + i];
-            l2v[e] = l == -CUDART_INF_F ? CUDART_INF_F : l * LOG2E;
-            dvv[e] = p.dvec[head_off + i];
+      int I = DYN ? (lane == 0 ? fetch_item<MODE>(p) : 0) : -1;
+      if (DYN) I = __shfl_sync(0xffffffffu, I, 0);
+      for (;;) {
+        if (DYN) {  // publish the item (or the end mark -1) to the other roles
+          const int rr = k % C::RING;
+          ok = wait_bar(ring_empty(rr), ((k / C::RING) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 3);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          if (lane == 0) {
+            ring[rr] = I;
+            bar_arrive(ring_full(rr));
+          }
+          ++k;
+          if (I < 0) break;
+        } else {
+          for (;;) {  // the static schedule, skipping empty items
+            I = bwd_item_index(k++);
+            if (I >= p.num_items || !item_of<MODE>(p, I).empty) break;
+          }
+          if (I >= p.num_items) break;
+        }
+        const BItem itm = item_of<MODE>(p, I);
+        int I_next = 0;
+        // K and V of this item once the previous item's products have read them
+        ok = wait_bar(kv_empty, (jn & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 2);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (lane == 0) {
+          bar_arrive_expect_tx(kv_full, 2 * C::TILE);
+          for (int c = 0; c < NCH; ++c) {
+            tma_load_4d(smem_u32(sK + c * 16384), &p.tm_k, kv_full, c * 64, itm.h, itm.trow + itm.k0, itm.bt);
+            tma_load_4d(smem_u32(sV + c * 16384), &p.tm_v, kv_full, c * 64, itm.h, itm.trow + itm.k0, itm.bt);
           }
         }
-        ok = wait_bar(q_empty(sq), ((it / QS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 0);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        float* side = sSide + sq * 256;
+        ++issued_kv;
+        // the next item's index: the atomic is in flight while this item loads
+        if (DYN && lane == 0) I_next = fetch_item<MODE>(p);
+        int qb = itm.qb_first;
+        for (int it = 0; it < itm.nq && ok; ++it, qb = next_qblock<MODE>(p, itm, qb)) {
+          const int gi = g + it;
+          const int i0 = (SPARSE ? qb : itm.qb_first + it) * 128;
+          const int sq = gi % QS;
+          // log2-scaled LSE and D of this query block, +inf / 0 past the end;
+          // loaded before waiting for the slot so the latency overlaps the wait
+          float l2v[4], dvv[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          // stored negated: the compute warps add them with paired FMAs
-          side[lane + 32 * e] = -l2v[e];
-          side[128 + lane + 32 * e] = -dvv[e];
+          for (int e = 0; e < 4; ++e) {
+            const int i = i0 + lane + 32 * e;
+            l2v[e] = CUDART_INF_F;
+            dvv[e] = 0.f;
+            if (i < itm.len) {
+              const float l = p.lse[itm.head_off + i];
+              l2v[e] = l == -CUDART_INF_F ? CUDART_INF_F : l * LOG2E;
+              dvv[e] = p.dvec[itm.head_off + i];
+            }
+          }
+          ok = wait_bar(q_empty(sq), ((gi / QS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 0);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          float* side = sSide + sq * 256;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            // stored negated: the compute warps add them with paired FMAs
+            side[lane + 32 * e] = -l2v[e];
+            side[128 + lane + 32 * e] = -dvv[e];
+          }
+          __threadfence_block();
+          __syncwarp();
+          if (lane == 0) {
+            bar_arrive_expect_tx(q_full(sq), C::TILE);
+            for (int c = 0; c < NCH; ++c)
+              tma_load_4d(smem_u32(sQ + sq * C::TILE + c * 16384), &p.tm_q, q_full(sq), c * 64, itm.h,
+                          itm.trow + i0, itm.bt);
+          }
+          ++issued_q;
+          const int sd = gi % DS;
+          ok = wait_bar(do_empty(sd), ((gi / DS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 1);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          if (lane == 0) {
+            bar_arrive_expect_tx(do_full(sd), C::TILE);
+            for (int c = 0; c < NCH; ++c)
+              tma_load_4d(smem_u32(sDO + sd * C::TILE + c * 16384), &p.tm_do, do_full(sd), c * 64, itm.h,
+                          itm.trow + i0, itm.bt);
+          }
+          ++issued_do;
         }
-        __threadfence_block();
-        __syncwarp();
-        if (lane == 0) {
-          bar_arrive_expect_tx(q_full(sq), C::TILE);
-          for (int c = 0; c < NCH; ++c)
-            tma_load_4d(smem_u32(sQ + sq * C::TILE + c * 16384), &p.tm_q, q_full(sq), c * 64, h, trow + i0,
-                        sv.bt);
-        }
-        ++issued_q;
-        const int sd = it % DS;
-        ok = wait_bar(do_empty(sd), ((it / DS) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 1);
-        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        if (lane == 0) {
-          bar_arrive_expect_tx(do_full(sd), C::TILE);
-          for (int c = 0; c < NCH; ++c)
-            tma_load_4d(smem_u32(sDO + sd * C::TILE + c * 16384), &p.tm_do, do_full(sd), c * 64, h,
-                        trow + i0, sv.bt);
+        g += itm.nq;
+        ++jn;
+        if (DYN) I = __shfl_sync(0xffffffffu, I_next, 0);
+      }
+      if (DYN && lane == 0) {
+        // The last CTA to finish taking items returns the counters to zero.
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+          p.sched[0] = 0u;
+          p.sched[1] = 0u;
+          __threadfence();
         }
-        ++issued_do;
       }
-      if (lane == 0) {
-        drain_wait(kv_full, 0, p.wait_ns);
-        for (int k = max(0, issued_q - QS); k < issued_q; ++k)
-          drain_wait(q_full(k % QS), (k / QS) & 1, p.wait_ns);
-        for (int k = max(0, issued_do - DS); k < issued_do; ++k)
-          drain_wait(do_full(k % DS), (k / DS) & 1, p.wait_ns);
+      if (lane == 0) {  // every copy issued must land before the CTA exits
+        if (issued_kv > 0) drain_wait(kv_full, (issued_kv - 1) & 1, p.wait_ns);
+        for (int q = max(0, issued_q - QS); q < issued_q; ++q)
+          drain_wait(q_full(q % QS), (q / QS) & 1, p.wait_ns);
+        for (int q = max(0, issued_do - DS); q < issued_do; ++q)
+          drain_wait(do_full(q % DS), (q / DS) & 1, p.wait_ns);
       }
-    } else if (warp == 13 && lane == 0) {
+    } else if (warp == 13) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t id_kq = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       const uint32_t id_pd = idesc_bf16_f32(128, HD, 0, 1);   // dV, dK (B MN-major)
@@ -369,13 +513,14 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           umma_ts(d_tmem, a_tmem + 64 * (kk / 4) + (kk % 4) * 8,
                   sdesc_sw128(bb + kk * 2048, 16384, 1024), id_pd, (acc || kk > 0) ? 1u : 0u);
       };
-      // Issue order.  Prologue: S_0, dP_0, dV_0, S_1.  Then for block i:
+      // Issue order.  Item prologue: S_0, dP_0, dV_0, S_1.  Then for block i:
       //   dK_i, dQ_i       (need dS_i)
       //   dP_{i+1}         (needs dQ_i drained out of the shared TMEM columns;
       //                     runs while the compute warps form P_{i+1})
       //   dV_{i+1}         (needs P_{i+1})
       //   S_{i+2}          (S columns are free once dV_{i+1} has read P_{i+1})
       // The compute warps work in the order P_0, dS_0, P_1, dS_1, ...
+      // Indices below are the CTA-wide query-block counter g + i.
       auto dp = [&](int k) {                      // dP_k^T = V dO_k^T
         const int sd = k % DS;
         if (!wait_bar(do_full(sd), (k / DS) & 1, ab, p.wait_ns, SITE_BMMA + 2)) return false;
@@ -402,221 +547,254 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         umma_commit(s_full);
         return true;
       };
-      bool ok = wait_bar(kv_full, 0, ab, p.wait_ns, SITE_BMMA + 0);
-      ok = ok && s_next(0);
-      ok = ok && dp(0);
-      ok = ok && dv(0, false);
-      if (ok && nq > 1) ok = s_next(1);
-      for (int it = 0; it < nq && ok; ++it) {
-        const int sq = it % QS;
-        ok = wait_bar(ds_ready, it & 1, ab, p.wait_ns, SITE_BMMA + 6);
-        if (!ok) break;
-        tc_fence_after();
-        from_tmem(tmem + T_DK, tmem + T_DP, sQ + sq * C::TILE, it > 0);   // dK += dS^T Q
-        umma_commit(q_empty(sq));
-        if (WITH_DQ) {
-          // dQ_i = dS K: A = dS (queries x keys) read MN-major from the dS^T
-          // tile, B = K (keys x d) MN-major.
-          const uint32_t a0 = smem_u32(sDS), kb0 = smem_u32(sK);
+      int jn = 0, g = 0, k = 0;
+      bool ok = true;
+      for (;;) {
+        int I;
+        if (lane == 0) ok = next_item(k, I, false, SITE_BMMA + 8);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        I = __shfl_sync(0xffffffffu, I, 0);
+        if (!ok || I < 0) break;
+        const BItem itm = item_of<MODE>(p, I);
+        const int nq = itm.nq;
+        if (lane == 0) {
+          ok = wait_bar(kv_full, jn & 1, ab, p.wait_ns, SITE_BMMA + 0);
+          ok = ok && s_next(g);
+          ok = ok && dp(g);
+          // dV_0 and dK_0 overwrite the accumulators: the compute warps must
+          // have read the previous item's
+          if (ok && jn > 0) ok = wait_bar(acc_empty, (jn - 1) & 1, ab, p.wait_ns, SITE_BMMA + 7);
+          ok = ok && dv(g, false);
+          if (ok && nq > 1) ok = s_next(g + 1);
+          for (int it = 0; it < nq && ok; ++it) {
+            const int gi = g + it;
+            const int sq = gi % QS;
+            ok = wait_bar(ds_ready, gi & 1, ab, p.wait_ns, SITE_BMMA + 6);
+            if (!ok) break;
+            tc_fence_after();
+            from_tmem(tmem + T_DK, tmem + T_DP, sQ + sq * C::TILE, it > 0);   // dK += dS^T Q
+            umma_commit(q_empty(sq));
+            if (WITH_DQ) {
+              // dQ_i = dS K: A = dS (queries x keys) read MN-major from the
+              // dS^T tile, B = K (keys x d) MN-major.
+              const uint32_t a0 = smem_u32(sDS), kb0 = smem_u32(sK);
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk)
-            umma_ss(tmem + T_DP, sdesc_sw128(a0 + kk * 2048, 16384, 1024),
-                    sdesc_sw128(kb0 + kk * 2048, 16384, 1024), id_dq, kk > 0);
-          umma_commit(dq_full);
+              for (int kk = 0; kk < 128 / 16; ++kk)
+                umma_ss(tmem + T_DP, sdesc_sw128(a0 + kk * 2048, 16384, 1024),
+                        sdesc_sw128(kb0 + kk * 2048, 16384, 1024), id_dq, kk > 0);
+              umma_commit(dq_full);
+            }
+            if (it + 1 < nq) ok = dp(gi + 1) && dv(gi + 1, true);
+            if (ok && it + 2 < nq) ok = s_next(gi + 2);
+          }
+          if (ok) {
+            umma_commit(kv_empty);   // every product reading K and V is issued
+            umma_commit(acc_full);
+          }
         }
-        if (it + 1 < nq) ok = dp(it + 1) && dv(it + 1, true);
-        if (ok && it + 2 < nq) ok = s_next(it + 2);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        g += nq;
+        ++jn;
       }
-      umma_commit(acc_full);
-      umma_commit(drain_bar);
-      drain_wait(drain_bar, 0, p.wait_ns);
+      if (lane == 0) {
+        umma_commit(drain_bar);
+        drain_wait(drain_bar, 0, p.wait_ns);
+      }
     }
   } else if (wg < 2) {
     regs_inc<C::REGS_COMPUTE>();
     // ------------------------------------------------------------ compute (key rows)
     const int r = (warp % 4) * 32 + lane;
-    const int j = k0 + r;
     const int cq = 64 * wg;  // this warpgroup's query columns [cq, cq + 64)
-    int lo_q = p.wr >= 0 ? max(0, j - p.wr) : 0;
-    int hi_q = p.wl >= 0 ? min(len - 1, j + p.wl) : len - 1;
-    if (j >= len) {
-      lo_q = 1;
-      hi_q = 0;
-    }
     const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
     const float C2 = p.scale_log2;
-    float slope2 = 0.f;
-    if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
+    int jn = 0, g = 0, k = 0;
     bool ok = true;
-    int qb = qb_first;
-    for (int it = 0; it < nq; ++it, qb = next_qb(qb)) {
-      const int i0 = (SPARSE ? qb : qb_first + it) * 128 + cq;
-      // a fully hidden block is visited only when the mask keeps none
-      const bool hidden = SPARSE && mcol[qb * p.nb] == 0;
-      const float* side = sSide + (it % QS) * 256 + cq;
-      ok = wait_bar(s_full, it & 1, ab, p.wait_ns, SITE_BCOMP + 0);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      float pr[64];
-      const bool full = (i0 >= lo_q) && (i0 + 63 <= hi_q);
-      const float fj = float(i0 - j);
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_base + T_S + cq + h2 * 32, u);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const int c = h2 * 32 + e;
-          const float4 l4 = *reinterpret_cast<const float4*>(side + c);  // -LSE log2(e)
-          float x0, x1, x2, x3;
-          if (ALIBI) {
-            x0 = fmaf(slope2, fabsf(fj + float(c)), fmaf(__uint_as_float(u[e]), C2, l4.x));
-            x1 = fmaf(slope2, fabsf(fj + float(c + 1)), fmaf(__uint_as_float(u[e + 1]), C2, l4.y));
-            x2 = fmaf(slope2, fabsf(fj + float(c + 2)), fmaf(__uint_as_float(u[e + 2]), C2, l4.z));
-            x3 = fmaf(slope2, fabsf(fj + float(c + 3)), fmaf(__uint_as_float(u[e + 3]), C2, l4.w));
-          } else {
-            const uint64_t c2x2 = pk2(C2, C2);
-            upk2(fma2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), c2x2, pk2(l4.x, l4.y)), x0, x1);
-            upk2(fma2(pk2(__uint_as_float(u[e + 2]), __uint_as_float(u[e + 3])), c2x2, pk2(l4.z, l4.w)), x2,
-                 x3);
-          }
-          pr[c] = ex2(x0);
-          pr[c + 1] = ex2(x1);
-          pr[c + 2] = ex2(x2);
-          pr[c + 3] = ex2(x3);
-        }
+    for (;;) {
+      int I;
+      ok = next_item(k, I, true, SITE_BCOMP + 3);
+      if (!ok || I < 0) break;
+      const BItem itm = item_of<MODE>(p, I);
+      const int h = itm.h, b = itm.b;
+      const int j = itm.k0 + r;
+      int lo_q = p.wr >= 0 ? max(0, j - p.wr) : 0;
+      int hi_q = p.wl >= 0 ? min(itm.len - 1, j + p.wl) : itm.len - 1;
+      if (j >= itm.len) {
+        lo_q = 1;
+        hi_q = 0;
       }
-      if (!full || hidden) {
+      float slope2 = 0.f;
+      if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
+      int qb = itm.qb_first;
+      for (int it = 0; it < itm.nq; ++it, qb = next_qblock<MODE>(p, itm, qb)) {
+        const int gi = g + it;
+        const int i0 = (SPARSE ? qb : itm.qb_first + it) * 128 + cq;
+        // a fully hidden block is visited only when the mask keeps none
+        const bool hidden = SPARSE && itm.mcol[qb * p.nb] == 0;
+        const float* side = sSide + (gi % QS) * 256 + cq;
+        ok = wait_bar(s_full, gi & 1, ab, p.wait_ns, SITE_BCOMP + 0);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        float pr[64];
+        const bool full = (i0 >= lo_q) && (i0 + 63 <= hi_q);
+        const float fj = float(i0 - j);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int i = i0 + c;
-          if (hidden || i < lo_q || i > hi_q) pr[c] = 0.f;
-        }
-      }
-      // Dropout: one generator call gives the bytes of four consecutive keys
-      // (a quad of lanes: k0 is a multiple of 128) for four consecutive
-      // queries; each lane computes one call in four and the quad trades.
-      uint32_t keep_lo = 0xFFFFFFFFu, keep_hi = 0xFFFFFFFFu;
-      if (DROPOUT) {
-        keep_lo = keep_hi = 0u;
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_base + T_S + cq + h2 * 32, u);
+          tmem_ld_wait();
 #pragma unroll
-        for (int t16 = 0; t16 < 4; ++t16) {
-          uint32_t z[4];
-          dropout_words_col16(p.drop, b, h, j, (i0 >> 2) + 4 * t16, z);
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t kept = dropout_keep(z[c4], e, p.drop.threshold) ? 1u : 0u;
-              const int c = 16 * t16 + 4 * c4 + e;
-              if (c < 32) keep_lo |= kept << c;
-              else keep_hi |= kept << (c - 32);
+          for (int e = 0; e < 32; e += 4) {
+            const int c = h2 * 32 + e;
+            const float4 l4 = *reinterpret_cast<const float4*>(side + c);  // -LSE log2(e)
+            float x0, x1, x2, x3;
+            if (ALIBI) {
+              x0 = fmaf(slope2, fabsf(fj + float(c)), fmaf(__uint_as_float(u[e]), C2, l4.x));
+              x1 = fmaf(slope2, fabsf(fj + float(c + 1)), fmaf(__uint_as_float(u[e + 1]), C2, l4.y));
+              x2 = fmaf(slope2, fabsf(fj + float(c + 2)), fmaf(__uint_as_float(u[e + 2]), C2, l4.z));
+              x3 = fmaf(slope2, fabsf(fj + float(c + 3)), fmaf(__uint_as_float(u[e + 3]), C2, l4.w));
+            } else {
+              const uint64_t c2x2 = pk2(C2, C2);
+              upk2(fma2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), c2x2, pk2(l4.x, l4.y)), x0,
+                   x1);
+              upk2(fma2(pk2(__uint_as_float(u[e + 2]), __uint_as_float(u[e + 3])), c2x2, pk2(l4.z, l4.w)),
+                   x2, x3);
             }
-        }
-      }
-      auto kept = [&](int c) {
-        return ((c < 32 ? keep_lo >> c : keep_hi >> (c - 32)) & 1u) != 0u;
-      };
-      // P^T (bf16, dropped and rescaled when dropout is on) into columns
-      // [cq, cq+32) of the S^T region (already read)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = c * 32 + 2 * e;
-          float a0 = pr[c0], a1 = pr[c0 + 1];
-          if (DROPOUT) {
-            a0 = kept(c0) ? a0 * p.drop.keep_scale : 0.f;
-            a1 = kept(c0 + 1) ? a1 * p.drop.keep_scale : 0.f;
+            pr[c] = ex2(x0);
+            pr[c + 1] = ex2(x1);
+            pr[c + 2] = ex2(x2);
+            pr[c + 3] = ex2(x3);
           }
-          w[e] = pack_bf16(a0, a1);
         }
-        tmem_st16(tmem + lane_base + T_S + cq + c * 16, w);
+        if (!full || hidden) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int i = i0 + c;
+            if (hidden || i < lo_q || i > hi_q) pr[c] = 0.f;
+          }
+        }
+        // Dropout: one generator call gives the bytes of four consecutive keys
+        // (a quad of lanes: k0 is a multiple of 128) for four consecutive
+        // queries; each lane computes one call in four and the quad trades.
+        uint32_t keep_lo = 0xFFFFFFFFu, keep_hi = 0xFFFFFFFFu;
+        if (DROPOUT) {
+          keep_lo = keep_hi = 0u;
+#pragma unroll
+          for (int t16 = 0; t16 < 4; ++t16) {
+            uint32_t z[4];
+            dropout_words_col16(p.drop, b, h, j, (i0 >> 2) + 4 * t16, z);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint32_t kept = dropout_keep(z[c4], e, p.drop.threshold) ? 1u : 0u;
+                const int c = 16 * t16 + 4 * c4 + e;
+                if (c < 32) keep_lo |= kept << c;
+                else keep_hi |= kept << (c - 32);
+              }
+          }
+        }
+        auto kept = [&](int c) {
+          return ((c < 32 ? keep_lo >> c : keep_hi >> (c - 32)) & 1u) != 0u;
+        };
+        // P^T (bf16, dropped and rescaled when dropout is on) into columns
+        // [cq, cq+32) of the S^T region (already read)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = c * 32 + 2 * e;
+            float a0 = pr[c0], a1 = pr[c0 + 1];
+            if (DROPOUT) {
+              a0 = kept(c0) ? a0 * p.drop.keep_scale : 0.f;
+              a1 = kept(c0 + 1) ? a1 * p.drop.keep_scale : 0.f;
+            }
+            w[e] = pack_bf16(a0, a1);
+          }
+          tmem_st16(tmem + lane_base + T_S + cq + c * 16, w);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        bar_arrive(p_ready);
+        // dS^T = P^T o (dP^T - D), 32 columns at a time
+        ok = wait_bar(dp_full, gi & 1, ab, p.wait_ns, SITE_BCOMP + 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_base + T_DP + cq + c * 32, u);
+          tmem_ld_wait();
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const int cc = c * 32 + 2 * e;
+            const float4 d4 = *reinterpret_cast<const float4*>(side + 128 + cc);  // -D
+            float g0 = __uint_as_float(u[2 * e]), g1 = __uint_as_float(u[2 * e + 1]);
+            float g2 = __uint_as_float(u[2 * e + 2]), g3 = __uint_as_float(u[2 * e + 3]);
+            if (DROPOUT) {  // dP = (dO V^T) o keep / (1 - p)
+              g0 = kept(cc) ? g0 * p.drop.keep_scale : 0.f;
+              g1 = kept(cc + 1) ? g1 * p.drop.keep_scale : 0.f;
+              g2 = kept(cc + 2) ? g2 * p.drop.keep_scale : 0.f;
+              g3 = kept(cc + 3) ? g3 * p.drop.keep_scale : 0.f;
+            }
+            float s0, s1, s2, s3;  // dS = P o (dP - D), two at a time
+            upk2(mul2(pk2(pr[cc], pr[cc + 1]), add2(pk2(g0, g1), pk2(d4.x, d4.y))), s0, s1);
+            upk2(mul2(pk2(pr[cc + 2], pr[cc + 3]), add2(pk2(g2, g3), pk2(d4.z, d4.w))), s2, s3);
+            w[e] = pack_bf16(s0, s1);
+            w[e + 1] = pack_bf16(s2, s3);
+          }
+          // written over columns this thread has already read
+          tmem_st16(tmem + lane_base + T_DP + cq + c * 16, w);
+          if (WITH_DQ) st_sw128_row32(sDS, r, cq + c * 32, w);
+        }
+        tmem_st_wait();
+        if (WITH_DQ) fence_proxy_async_smem();
+        tc_fence_before();
+        bar_arrive(ds_ready);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      bar_arrive(p_ready);
-      // dS^T = P^T o (dP^T - D), 32 columns at a time
-      ok = wait_bar(dp_full, it & 1, ab, p.wait_ns, SITE_BCOMP + 1);
+      if (!ok) break;
+      // -------------------------------------------------------- item epilogue
+      // This warpgroup's half of the d columns of dV and dK leaves TMEM into
+      // registers (then the accumulators are free for the next item) and
+      // goes to global memory as 16-byte row stores; the rows of a key block
+      // that runs past the end of a packed sequence are not written.
+      ok = wait_bar(acc_full, jn & 1, ab, p.wait_ns, SITE_BCOMP + 2);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      constexpr int NC = HD / 64;  // 32-column chunks per warpgroup and tensor
+      uint32_t wv[NC][16], wk[NC][16];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < NC; ++c) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_base + T_DP + cq + c * 32, u);
-        tmem_ld_wait();
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const int cc = c * 32 + 2 * e;
-          const float4 d4 = *reinterpret_cast<const float4*>(side + 128 + cc);  // -D
-          float g0 = __uint_as_float(u[2 * e]), g1 = __uint_as_float(u[2 * e + 1]);
-          float g2 = __uint_as_float(u[2 * e + 2]), g3 = __uint_as_float(u[2 * e + 3]);
-          if (DROPOUT) {  // dP = (dO V^T) o keep / (1 - p)
-            g0 = kept(cc) ? g0 * p.drop.keep_scale : 0.f;
-            g1 = kept(cc + 1) ? g1 * p.drop.keep_scale : 0.f;
-            g2 = kept(cc + 2) ? g2 * p.drop.keep_scale : 0.f;
-            g3 = kept(cc + 3) ? g3 * p.drop.keep_scale : 0.f;
-          }
-          float s0, s1, s2, s3;  // dS = P o (dP - D), two at a time
-          upk2(mul2(pk2(pr[cc], pr[cc + 1]), add2(pk2(g0, g1), pk2(d4.x, d4.y))), s0, s1);
-          upk2(mul2(pk2(pr[cc + 2], pr[cc + 3]), add2(pk2(g2, g3), pk2(d4.z, d4.w))), s2, s3);
-          w[e] = pack_bf16(s0, s1);
-          w[e + 1] = pack_bf16(s2, s3);
-        }
-        // written over columns this thread has already read
-        tmem_st16(tmem + lane_base + T_DP + cq + c * 16, w);
-        if (WITH_DQ) st_sw128_row32(sDS, r, cq + c * 32, w);
-      }
-      tmem_st_wait();
-      if (WITH_DQ) fence_proxy_async_smem();
-      tc_fence_before();
-      bar_arrive(ds_ready);
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok) ok = wait_bar(acc_full, 0, ab, p.wait_ns, SITE_BCOMP + 2);
-    ok = __all_sync(0xffffffffu, ok);
-    tc_fence_after();
-    // A whole tile leaves by TMA store; a tile whose last rows belong to the
-    // next packed sequence is written row by row instead.  (The sequence's
-    // rows are looked up again here rather than kept live through the loop.)
-    const SeqView so = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};
-    const bool tile_store = !PACKED || k0 + 128 <= so.len;
-    if (ok) {
-      // this warpgroup's half of the d columns of dV and dK -> bf16 -> the
-      // V and K tiles (free now) -> TMA store
-#pragma unroll
-      for (int c = 0; c < HD / 64; ++c) {
-        const int col = wg * (HD / 2) + c * 32;
-        uint32_t u[32], w[16];
-        tmem_ld32(tmem + lane_base + T_DV + col, u);
+        tmem_ld32(tmem + lane_base + T_DV + wg * (HD / 2) + c * 32, u);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) w[e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
-        if (tile_store) st_sw128_row32(sV, r, col, w);
-        else if (j < so.len) st_global_row32(p.dv, p.sdv, so, j, h, col, w);
-        tmem_ld32(tmem + lane_base + T_DK + col, u);
+        for (int e = 0; e < 16; ++e) wv[c][e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+        tmem_ld32(tmem + lane_base + T_DK + wg * (HD / 2) + c * 32, u);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16(__uint_as_float(u[2 * e]) * p.scale, __uint_as_float(u[2 * e + 1]) * p.scale);
-        if (tile_store) st_sw128_row32(sK, r, col, w);
-        else if (j < so.len) st_global_row32(p.dk, p.sdk, so, j, h, col, w);
+          wk[c][e] = pack_bf16(__uint_as_float(u[2 * e]) * p.scale, __uint_as_float(u[2 * e + 1]) * p.scale);
       }
-    }
-    fence_proxy_async_smem();
-    named_bar_sync(1, 256);
-    if (ok && tile_store && threadIdx.x == 0) {
-      for (int c = 0; c < NCH; ++c) {
-        tma_store_4d(&p.tm_dv, smem_u32(sV + c * 16384), c * 64, h, so.row0 + k0, so.bt);
-        tma_store_4d(&p.tm_dk, smem_u32(sK + c * 16384), c * 64, h, so.row0 + k0, so.bt);
+      tc_fence_before();
+      bar_arrive(acc_empty);
+      const SeqView so{itm.bt, itm.trow, itm.len};
+      if (j < itm.len) {
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          const int col = wg * (HD / 2) + c * 32;
+          st_global_row32(p.dv, p.sdv, so, j, h, col, wv[c]);
+          st_global_row32(p.dk, p.sdk, so, j, h, col, wk[c]);
+        }
       }
-      bulk_commit();
-      bulk_wait_all();
+      g += itm.nq;
+      ++jn;
     }
   } else {
     regs_inc<C::REGS_DRAIN>();
@@ -624,48 +802,68 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       // ---------------------------------------------------------- dQ drain (query rows)
       const int q = (warp % 4) * 32 + lane;
       const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
-      const int bh = sv.bt * p.H + h;
-      int qb = qb_first;
-      for (int it = 0; it < nq; ++it, qb = next_qb(qb)) {
-        const int i0 = (SPARSE ? qb : qb_first + it) * 128;
-        bool ok = wait_bar(dq_full, it & 1, ab, p.wait_ns, SITE_BRED);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after();
-        // dQ leaves TMEM 32 columns (one 128-byte swizzled box of 128 rows)
-        // at a time and is added into the accumulator with one TMA bulk
-        // reduction per box, staged through a two-slot ring.  Chunks 0..1
-        // go out right away; the remaining chunks are read into registers
-        // before TMEM is released, then staged as their slots free up.
-        // Each warp stages its own 32 rows (a 32 x 32-column box, 4 KB) and
-        // issues the bulk reduction for them: no cross-warp barrier.
-        const int wq = warp % 4;
-        auto stage = [&](const uint32_t (&u)[32], int chunk) {
-          if (lane == 0) bulk_wait_read_1();   // this warp's previous box in the slot was read
-          __syncwarp();
-          uint8_t* row = sStg + (chunk & 1) * 16384 + q * 128;
+      const int wq = warp % 4;
+      int g = 0, k = 0;
+      bool ok = true;
+      for (;;) {
+        int I;
+        ok = next_item(k, I, true, SITE_BRED + 1);
+        if (!ok || I < 0) break;
+        const BItem itm = item_of<MODE>(p, I);
+        const int bh = itm.bt * p.H + itm.h;
+        int qb = itm.qb_first;
+        for (int it = 0; it < itm.nq; ++it, qb = next_qblock<MODE>(p, itm, qb)) {
+          const int gi = g + it;
+          const int i0 = (SPARSE ? qb : itm.qb_first + it) * 128;
+          ok = wait_bar(dq_full, gi & 1, ab, p.wait_ns, SITE_BRED);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          // dQ leaves TMEM 32 columns (one 128-byte swizzled box of 128 rows)
+          // at a time and is added into the accumulator with one TMA bulk
+          // reduction per box, staged through a two-slot ring.  The whole tile
+          // is read into registers before TMEM is released, then staged as
+          // the slots free up.  Each warp stages its own 32 rows (a 32 x
+          // 32-column box, 4 KB) and issues the bulk reduction for them: no
+          // cross-warp barrier.
+          auto stage = [&](const uint32_t (&u)[32], int chunk) {
+            if (lane == 0) bulk_wait_read_1();   // this warp's previous box in the slot was read
+            __syncwarp();
+            uint8_t* row = sStg + (chunk & 1) * 16384 + q * 128;
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            *reinterpret_cast<uint4*>(row + ((e ^ (q & 7)) * 16)) =
-                make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sStg + (chunk & 1) * 16384 + wq * 4096), chunk * 32,
-                              trow + i0 + wq * 32, bh);
-            bulk_commit();
-          }
-        };
-        constexpr int NC = HD / 32;
-        uint32_t u[NC][32];
+            for (int e = 0; e < 8; ++e)
+              *reinterpret_cast<uint4*>(row + ((e ^ (q & 7)) * 16)) =
+                  make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sStg + (chunk & 1) * 16384 + wq * 4096), chunk * 32,
+                                itm.trow + i0 + wq * 32, bh);
+              bulk_commit();
+            }
+          };
+          constexpr int NC = HD / 32;
+          uint32_t u[NC][32];
 #pragma unroll
-        for (int c = 0; c < NC; ++c) tmem_ld32(tmem + lane_base + T_DP + c * 32, u[c]);
-        tmem_ld_wait();
-        tc_fence_before();
-        bar_arrive(dq_free);   // TMEM columns may now take the next dP^T
+          for (int c = 0; c < NC; ++c) tmem_ld32(tmem + lane_base + T_DP + c * 32, u[c]);
+          tmem_ld_wait();
+          tc_fence_before();
+          bar_arrive(dq_free);   // TMEM columns may now take the next dP^T
 #pragma unroll
-        for (int c = 0; c < NC; ++c) stage(u[c], c);
+          for (int c = 0; c < NC; ++c) stage(u[c], c);
+        }
+        if (!ok) break;
+        g += itm.nq;
       }
       if (lane == 0) bulk_wait_all();
+    } else if (DYN) {
+      // without dQ this warpgroup still takes its ring entries, so the
+      // loader can reuse them
+      int k = 0;
+      for (;;) {
+        int I;
+        if (!next_item(k, I, true, SITE_BRED + 2) || I < 0) break;
+      }
     }
   }
 

@@ -42,8 +42,10 @@ fa2_status check_shape(int B, int N, int H, int d, fa2_dtype dtype) {
   if (dtype != FA2_BF16 && dtype != FA2_F32) return FA2_ERR_INVALID_ARG;
   // grid limits of the launches below
   if (B > 65535 || H > 65535) return FA2_ERR_INVALID_ARG;
-  const long long pairs = (N + 255) / 256;
-  if (pairs * H * B > 0x7fffffffLL) return FA2_ERR_INVALID_ARG;
+  // key blocks x heads x batch (the backward's work items, walked by a
+  // persistent grid with int indices) must stay well inside int
+  const long long blocks = (N + 127) / 128;
+  if (blocks * H * B > 0x7fff0000LL) return FA2_ERR_INVALID_ARG;
   if ((long long)B * H * N > (1LL << 40)) return FA2_ERR_INVALID_ARG;
   return FA2_OK;
 }
@@ -354,6 +356,15 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.wait_ns = g_wait_ns.load();
   p.drop = a.drop;
   const unsigned grid = unsigned(p.nblocks) * unsigned(a.H) * unsigned(a.B);
+  // kernel 1 is persistent: one CTA per SM walks the work items
+  p.num_items = int(grid);
+  DeviceInfo di;
+  {
+    int dev2;
+    FA2_TRY(current_device(&dev2, &di));
+  }
+  const unsigned grid1 = std::min<unsigned>(grid, unsigned(std::max(di.sm_count, 1)));
+  if (MODE != kLayoutPadded) FA2_TRY(sched_counters(dev, &p.sched));
   constexpr int smem1 = BwdCfg<HD>::SMEM_BYTES;
   // Kernel 1 re-balances registers between its warpgroups; the shares add up
   // to 512 threads x REGS_AT_LAUNCH, so the compiled kernel must launch with
@@ -373,7 +384,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
     FA2_TRY(launched(1));
     auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE>;
     FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv));
-    k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
+    k1<<<grid1, BwdCfg<HD>::THREADS, smem1, st>>>(p);
     FA2_TRY(launched(1));
     AttnArgs c = a;  // the accumulator is [bt * H, rows, d] in both layouts
     c.B = ms.bt;
@@ -386,7 +397,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   }
   auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, MODE>;
   FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv_nodq));
-  k1<<<grid, BwdCfg<HD>::THREADS, smem1, st>>>(p);
+  k1<<<grid1, BwdCfg<HD>::THREADS, smem1, st>>>(p);
   FA2_TRY(launched(1));
   auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI, DROPOUT, MODE>;
   constexpr int smem2 = DqCfg<HD>::SMEM_BYTES;
