@@ -348,9 +348,6 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.wl = a.wl;
   p.wr = a.wr;
   p.nblocks = (a.N + 127) / 128;
-  // key blocks of one head next to each other (they share its Q and dO in
-  // L2) unless masks make the blocks' work vary
-  p.heavy_first = (a.wr >= 0 || a.wl >= 0) ? 1 : 0;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.wait_ns = g_wait_ns.load();
