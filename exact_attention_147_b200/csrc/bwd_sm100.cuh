@@ -7,11 +7,11 @@
 //     P  = exp(c S - LSE),   dV = P^T dO,   dP = dO V^T,
 //     dS = P o (dP - D),     dK = c dS^T Q,  dQ = c dS K.
 //
-// Kernel 1, fa2_bwd_dkdv_sm100_kernel: one CTA per 128-key block of one
-// (batch, head), parallel over key blocks (FlashAttention-2 abstract: work
-// split across thread blocks even within a head).  K_j and V_j stay in shared
-// memory; the query blocks that see them stream through a TMA ring.  Per query
-// block, with keys on the TMEM lanes:
+// Kernel 1, fa2_bwd_dkdv_sm100_kernel: parallel over 128-key blocks of each
+// (batch, head) (FlashAttention-2 abstract: work split across thread blocks
+// even within a head); a persistent grid of one CTA per SM walks these key
+// blocks.  K_j and V_j stay in shared memory; the query blocks that see them
+// stream through a TMA ring.  Per query block, with keys on the TMEM lanes:
 //     S^T  = K Q^T          (tcgen05, SS)       -> TMEM [0,128)
 //     dP^T = V dO^T         (tcgen05, SS)       -> TMEM [128,256)
 //     P^T  = exp2(S^T c log2e - LSE log2e)       (compute warps, -> bf16 over S^T)
@@ -21,7 +21,7 @@
 //     dK  += dS^T Q         (tcgen05, A from TMEM)
 //     dQ_i = dS K           (tcgen05, A = dS from shared memory, MN-major)
 //                           -> TMEM [128,128+d), added into an fp32 dQ
-//                              accumulator in global memory with vector
+//                              accumulator in global memory with TMA bulk
 //                              reductions (order of the adds is not fixed).
 // With `deterministic`, kernel 1 skips dQ and kernel 2 produces it.
 //
