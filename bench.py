@@ -382,6 +382,8 @@ def run_gpu(args):
         line["packed"] = run_packed(F, W)
         line["blocksparse"] = run_blocksparse(F, W)
         line["fp8"] = run_fp8(F, W)
+        line["long_local"] = run_long_local(F, W)
+        line["alibi_det"] = run_alibi_det(F, W)
     if rank == 0:
         print(json.dumps(line), flush=True)
     ranks.finalize(world)
@@ -537,6 +539,72 @@ def run_fp8(F, W):
                     "frac_of_e4m3_peak": round(tfl / fp8_peak, 3),
                     "e4m3_peak": f"2 x {src} bf16_tflops = {fp8_peak:.0f}"})
         del q8, k8, v8, out, lse
+    return res
+
+
+def allowed_pairs(N, causal, wl, wr):
+    """Number of visible (query, key) pairs of one head: the FLOP count of a
+    windowed call is 4 d per pair (x 2.5 for the backward)."""
+    total = 0
+    for i in range(N):
+        lo = max(0, i - wl) if wl >= 0 else 0
+        hi = i if causal else (min(N - 1, i + wr) if wr >= 0 else N - 1)
+        total += hi - lo + 1
+    return total
+
+
+def run_long_local(F, W):
+    """B=1, H=32, N=32768, d=128, causal, window (4096, 0): fwd and bwd timed
+    apart; FLOPs count the visible pairs only."""
+    import torch
+    w = W.long_local()
+    q, k, v, do = W.make_inputs(w, "cuda")
+    win = (w.window_left, w.window_right)
+    out, lse = F.fwd(q, k, v, causal=True, window_size=win)
+    D = F.bwd_preprocess(out, do)
+    dq, dk, dv = F.bwd(do, q, k, v, lse, D, causal=True, window_size=win)
+    ws = torch.empty(F.workspace_size(w.B, w.N, w.H, w.d, torch.bfloat16), dtype=torch.uint8,
+                     device="cuda")
+    tf, tb = _time_pair(lambda: F.fwd(q, k, v, causal=True, window_size=win, out=out, lse=lse),
+                        lambda: F.bwd(do, q, k, v, lse, D, causal=True, window_size=win, dq=dq, dk=dk,
+                                      dv=dv, workspace=ws), reps=5)
+    ff = 4.0 * w.B * w.H * w.d * allowed_pairs(w.N, True, w.window_left, w.window_right)
+    res = {"workload": "B=1 H=32 N=32768 d=128 causal window (4096, 0)", "flops_fwd": ff,
+           "fwd_ms": round(tf, 4), "fwd_tflops": round(ff / (tf * 1e-3) / 1e12, 1),
+           "bwd_ms": round(tb, 4), "bwd_tflops": round(2.5 * ff / (tb * 1e-3) / 1e12, 1)}
+    del q, k, v, do, out, lse, D, dq, dk, dv, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_alibi_det(F, W):
+    """B=4, H=16, N=4096, d=128, causal, ALiBi: forward, deterministic backward
+    (whose ordered dQ pass recomputes S, P and dS: that work is not counted)
+    and, beside it, the atomic backward; plus a bitwise repeat check."""
+    import torch
+    w = W.alibi_det()
+    q, k, v, do = W.make_inputs(w, "cuda")
+    sl = w.alibi_slopes().cuda()
+    out, lse = F.fwd(q, k, v, causal=True, alibi_slopes=sl)
+    D = F.bwd_preprocess(out, do)
+    grads = [F.bwd(do, q, k, v, lse, D, causal=True, alibi_slopes=sl, deterministic=True) for _ in range(2)]
+    repeat = all(torch.equal(a, b) for a, b in zip(grads[0], grads[1]))
+    dq, dk, dv = grads[0]
+    ws = {det: torch.empty(max(1, F.workspace_size(w.B, w.N, w.H, w.d, torch.bfloat16, det)),
+                           dtype=torch.uint8, device="cuda") for det in (False, True)}
+    bwd = {det: (lambda det=det: F.bwd(do, q, k, v, lse, D, causal=True, alibi_slopes=sl, deterministic=det,
+                                       dq=dq, dk=dk, dv=dv, workspace=ws[det])) for det in (False, True)}
+    tf, tb_det = _time_pair(lambda: F.fwd(q, k, v, causal=True, alibi_slopes=sl, out=out, lse=lse), bwd[True])
+    _, tb = _time_pair(lambda: None, bwd[False])
+    ff = flops_fwd(w.B, w.H, w.N, w.d, True)
+    res = {"workload": "B=4 H=16 N=4096 d=128 causal ALiBi", "fwd_ms": round(tf, 4),
+           "fwd_tflops": round(ff / (tf * 1e-3) / 1e12, 1),
+           "bwd_deterministic_ms": round(tb_det, 4),
+           "bwd_deterministic_tflops": round(2.5 * ff / (tb_det * 1e-3) / 1e12, 1),
+           "bwd_atomic_ms": round(tb, 4), "bwd_atomic_tflops": round(2.5 * ff / (tb * 1e-3) / 1e12, 1),
+           "deterministic_bitwise_repeat": bool(repeat)}
+    del q, k, v, do, out, lse, D, dq, dk, dv, ws, grads
+    torch.cuda.empty_cache()
     return res
 
 

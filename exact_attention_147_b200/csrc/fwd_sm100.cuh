@@ -30,6 +30,11 @@
 // P is written back over S and fed to the PV product straight from TMEM.
 // The tensor-core pipe runs its instructions in issue order, so S_t of the
 // next block may be issued right after the PV product that still reads P_t.
+// At d = 64 the O tiles leave 128 columns free and P_t gets its own 64
+// ([384 + 64t, 448 + 64t)): S_t of the next block is then issued as soon as
+// the softmax has read S_t into registers, and runs while the softmax is
+// still working on the current block, so a softmax warpgroup never waits for
+// the tensor cores between blocks.
 //
 // Online softmax (explainer "AI基础 | Flash Attention", "Online softmax"):
 // each thread keeps its row's running max m and running sum l in registers
@@ -100,9 +105,13 @@ struct FwdCfg {
   static constexpr int OFF_KV = QBUFS * NQT * QT_BYTES;
   static constexpr int OFF_BARS = OFF_KV + SLOTS * KV_BYTES;
   static constexpr int RING = 4;        // unit-index ring of the packed scheduler
+  // d = 64 leaves 128 TMEM columns free: P gets its own 64 columns per tile,
+  // so the next S product need not wait for the PV product that reads P.
+  static constexpr bool PSEP = HD == 64 && !FP8;
   // q_full[2], q_empty[2], slot full/empty, s_full[2], p_ready[2], o_full[2],
-  // o_empty[2], drain, ring full[4], ring empty[4], stats_full[2], stats_free[2]
-  static constexpr int NBARS = 2 * QBUFS + 2 * SLOTS + 4 * NQT + 1 + 2 * RING + 2 * NQT;
+  // o_empty[2], drain, ring full[4], ring empty[4], stats_full[2], stats_free[2],
+  // s_read[2], p_free[2]
+  static constexpr int NBARS = 2 * QBUFS + 2 * SLOTS + 4 * NQT + 1 + 2 * RING + 4 * NQT;
   // barriers, then the TMEM address, the abort flag, 2 spare words, the ring
   // and the per-row results (1 / l, LSE) the softmax hands to the epilogue
   static constexpr int OFF_STATS = OFF_BARS + NBARS * 8 + 16 + 4 * RING;
@@ -111,7 +120,9 @@ struct FwdCfg {
   static constexpr int THREADS = 512;
   // registers per thread after re-balancing (launch: 128 x 512 = 65536):
   // softmax warpgroups 184, epilogue warpgroup 80, loader / MMA warpgroup 64
-  static constexpr int REGS_SOFT = HD == 128 ? 184 : 176, REGS_EPI = 80, REGS_MISC = HD == 128 ? 64 : 80;
+  // (d = 64: 200 / 56 / 56, the split at which none of the roles spills)
+  static constexpr int REGS_SOFT = HD == 128 ? 184 : 200, REGS_EPI = HD == 128 ? 80 : 56,
+                       REGS_MISC = HD == 128 ? 64 : 56;
   static constexpr int REGS_AT_LAUNCH = (2 * 128 * REGS_SOFT + 128 * REGS_EPI + 128 * REGS_MISC) / 512;
   static_assert(REGS_AT_LAUNCH == 128, "register split must use exactly the launch budget");
 };
@@ -260,6 +271,9 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
   constexpr int BM = C::BM, BN = C::BN, NQT = C::NQT, SLOTS = C::SLOTS;
   constexpr int NCH = HD * C::ESZ / 128;  // 128-byte boxes per tile row
   constexpr int KSTEP = C::KSTEP;
+  // TMEM column of P_t: over S_t, or (separate-P layout) after the O tiles
+  constexpr int P_COL = C::PSEP ? 256 + NQT * HD : 0, P_STRIDE = C::PSEP ? BN / 2 : 128;
+  static_assert(!C::PSEP || P_COL + NQT * P_STRIDE <= 512, "tensor memory budget");
   using namespace fwd_detail;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -284,6 +298,9 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
   auto ring_empty = [&](int r) { return bar0 + 8u * (13 + 2 * SLOTS + C::RING + r); };
   auto stats_full = [&](int t) { return bar0 + 8u * (13 + 2 * SLOTS + 2 * C::RING + t); };
   auto stats_free = [&](int t) { return bar0 + 8u * (15 + 2 * SLOTS + 2 * C::RING + t); };
+  // separate-P layout only: S_t has been read into registers / P_t has been read by its PV product
+  auto s_read = [&](int t) { return bar0 + 8u * (17 + 2 * SLOTS + 2 * C::RING + t); };
+  auto p_free = [&](int t) { return bar0 + 8u * (19 + 2 * SLOTS + 2 * C::RING + t); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* ring = abort_flag + 3;  // packed: unit indices handed from the producer to the other roles
@@ -300,6 +317,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
       if (bar == p_ready(0) || bar == p_ready(1) || bar == o_empty(0) || bar == o_empty(1)) cnt = 128;
       if (bar == stats_full(0) || bar == stats_full(1) || bar == stats_free(0) || bar == stats_free(1))
         cnt = 128;
+      if (bar == s_read(0) || bar == s_read(1)) cnt = 128;
       // MMA + 8 softmax warps + 4 epilogue warps
       if (bar >= ring_empty(0) && bar <= ring_empty(C::RING - 1)) cnt = 13;
       bar_init(bar, cnt);
@@ -411,9 +429,11 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         for (int kk = 0; kk < BN / KSTEP; ++kk) {
           const uint64_t vd = sdesc_sw128(v0 + kk * KSTEP * 128, BN * 128, 1024);
           if (FP8)
-            umma_ts_f8(tmem + 256 + t * HD, tmem + t * 128 + kk * 8, vd, id_pv, (acc || kk > 0) ? 1u : 0u);
+            umma_ts_f8(tmem + 256 + t * HD, tmem + P_COL + t * P_STRIDE + kk * 8, vd, id_pv,
+                       (acc || kk > 0) ? 1u : 0u);
           else
-            umma_ts(tmem + 256 + t * HD, tmem + t * 128 + kk * 8, vd, id_pv, (acc || kk > 0) ? 1u : 0u);
+            umma_ts(tmem + 256 + t * HD, tmem + P_COL + t * P_STRIDE + kk * 8, vd, id_pv,
+                    (acc || kk > 0) ? 1u : 0u);
         }
       };
       int n = 0, g = 0;  // KV slots, blocks
@@ -435,6 +455,54 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         const int qb = k & 1;
         ok = wait_bar(q_full(qb), (k >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
         if (!ok) break;
+        if constexpr (C::PSEP) {
+          // Step it issues S_t of block it as soon as softmax t has read the
+          // previous S_t, then PV_t of block it-1 once P_t is ready: each
+          // softmax warpgroup finds its next S finished when it completes a
+          // block.  K of block it sits in slot n + 2 it, V in the next one.
+          for (int it = 0; it <= u.nblk && ok; ++it) {
+            const int gi = g + it;
+            const int nk = n + 2 * it, nv = nk - 1;
+            if (it < u.nblk) {
+              ok = wait_bar(slot_full(nk % SLOTS), (nk / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
+              if (!ok) break;
+            }
+            if (it > 0) {
+              ok = wait_bar(slot_full(nv % SLOTS), (nv / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
+              if (!ok) break;
+            }
+            for (int t = 0; t < NQT && ok; ++t) {
+              if (it < u.nblk) {
+                if (gi > 0) ok = wait_bar(s_read(t), (gi - 1) & 1, ab, p.wait_ns, SITE_MMA + 9);
+                if (!ok) break;
+                tc_fence_after();
+                qk(t, qb, nk % SLOTS);
+                umma_commit(s_full(t));
+              }
+              if (it > 0) {
+                ok = wait_bar(p_ready(t), (gi - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
+                // the first PV of a unit overwrites O_t: the previous unit's
+                // epilogue must have read it
+                if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+                if (!ok) break;
+                tc_fence_after();
+                pv(t, nv % SLOTS, it > 1);
+                umma_commit(p_free(t));
+                if (it == u.nblk) umma_commit(o_full(t));
+              }
+            }
+            if (!ok) break;
+            if (it < u.nblk) {
+              umma_commit(slot_empty(nk % SLOTS));
+              if (it == u.nblk - 1) umma_commit(q_empty(qb));  // the unit's last S products
+            }
+            if (it > 0) umma_commit(slot_empty(nv % SLOTS));
+          }
+          if (!ok) break;
+          n += 2 * u.nblk;
+          g += u.nblk;
+          continue;
+        }
         {
           const int sk = n % SLOTS;
           ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
@@ -566,6 +634,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
     const int r = (warp % 4) * 32 + lane;
     const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
     const uint32_t s_addr = tmem + lane_base + t * 128;
+    const uint32_t p_addr = tmem + lane_base + P_COL + t * P_STRIDE;
     const uint32_t o_addr = tmem + lane_base + 256 + t * HD;
     const float C2 = p.scale_log2;
     int g = 0;
@@ -613,6 +682,10 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
           for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(w32[e]);
         }
         tmem_ld_wait();
+        if (C::PSEP) {  // S_t is in registers: its columns may take the next block's S
+          tc_fence_before();
+          bar_arrive(s_read(t));
+        }
         if (ALIBI) {
           const float fi = float(i - kv0);
 #pragma unroll
@@ -661,6 +734,13 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         upk2(add2(l2x[0], l2x[1]), la, lb);
         upk2(add2(l2x[2], l2x[3]), lc, ld);
         l_run = fmaf(l_run, alpha, (la + lb) + (lc + ld));
+        if (C::PSEP && g + it > 0) {
+          // P_t and O_t are free once the previous block's PV product is done
+          ok = wait_bar(p_free(t), (g + it - 1) & 1, ab, p.wait_ns, SITE_SOFT + 6);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+        }
         // P (bf16 pairs) over the first BN/2 columns of S.  With dropout, l
         // keeps the un-dropped sum and dropped probabilities leave P here:
         // one generator call per quad of rows and 16 keys (the rows of a quad
@@ -675,7 +755,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             for (int e = 0; e < 16; ++e)
               w16[e] = pack_e4m3x4(s[c * 64 + 4 * e], s[c * 64 + 4 * e + 1], s[c * 64 + 4 * e + 2],
                                    s[c * 64 + 4 * e + 3]);
-            tmem_st16(s_addr + c * 16, w16);
+            tmem_st16(p_addr + c * 16, w16);
           }
         }
 #pragma unroll
@@ -696,10 +776,11 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
               }
             }
           }
-          tmem_st16(s_addr + c * 16, w16);
+          tmem_st16(p_addr + c * 16, w16);
         }
         // Rescale the running output (the PV product of the previous block has
-        // completed: S_t of this block was committed after it).
+        // completed: S_t of this block was committed after it, or, with the
+        // separate-P layout, p_free said so).
         if (it > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
