@@ -436,164 +436,230 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
                     (acc || kk > 0) ? 1u : 0u);
         }
       };
-      // The k-th unit: the loader's ring entry or the static schedule; -1
-      // past the last unit, -2 when the wait for the ring gave up.
-      auto fetch = [&](int k) -> int {
-        if (DYN) {
-          const int r = k % C::RING;
-          if (!wait_bar(ring_full(r), (k / C::RING) & 1, ab, p.wait_ns, SITE_MMA + 8)) return -2;
-          const int L = ring[r];
-          bar_arrive(ring_empty(r));
-          return L < 0 ? -1 : L;
-        }
-        const int L = unit_index(k);
-        return L >= p.num_units ? -1 : L;
-      };
-      int n = 0, g = 0;  // KV slots, blocks
-      bool ok = true;
-      // this unit's first S products went out with the previous unit's last
-      // PV products (every unit but the first; not in the separate-P layout)
-      bool s0_issued = false;
-      int L = fetch(0);
-      for (int k = 0; ok && L >= 0; ++k) {
-        const Unit u = unit_of<MODE>(p, L);
-        const int qb = k & 1;
-        if (!s0_issued) {
+      if constexpr (DYN || C::PSEP) {
+        int n = 0, g = 0;  // KV slots, blocks
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+          int L;
+          if (DYN) {
+            const int r = k % C::RING;
+            ok = wait_bar(ring_full(r), (k / C::RING) & 1, ab, p.wait_ns, SITE_MMA + 8);
+            if (!ok) break;
+            L = ring[r];
+            bar_arrive(ring_empty(r));
+            if (L < 0) break;
+          } else {
+            L = unit_index(k);
+            if (L >= p.num_units) break;
+          }
+          const Unit u = unit_of<MODE>(p, L);
+          const int qb = k & 1;
           ok = wait_bar(q_full(qb), (k >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
           if (!ok) break;
-        }
-        if constexpr (C::PSEP) {
-          // Step it issues S_t of block it as soon as softmax t has read the
-          // previous S_t, then PV_t of block it-1 once P_t is ready: each
-          // softmax warpgroup finds its next S finished when it completes a
-          // block.  K of block it sits in slot n + 2 it, V in the next one.
-          for (int it = 0; it <= u.nblk && ok; ++it) {
-            const int gi = g + it;
-            const int nk = n + 2 * it, nv = nk - 1;
-            if (it < u.nblk) {
-              ok = wait_bar(slot_full(nk % SLOTS), (nk / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
-              if (!ok) break;
-            }
-            if (it > 0) {
-              ok = wait_bar(slot_full(nv % SLOTS), (nv / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
-              if (!ok) break;
-            }
-            for (int t = 0; t < NQT && ok; ++t) {
+          if constexpr (C::PSEP) {
+            // Step it issues S_t of block it as soon as softmax t has read the
+            // previous S_t, then PV_t of block it-1 once P_t is ready: each
+            // softmax warpgroup finds its next S finished when it completes a
+            // block.  K of block it sits in slot n + 2 it, V in the next one.
+            for (int it = 0; it <= u.nblk && ok; ++it) {
+              const int gi = g + it;
+              const int nk = n + 2 * it, nv = nk - 1;
               if (it < u.nblk) {
-                if (gi > 0) ok = wait_bar(s_read(t), (gi - 1) & 1, ab, p.wait_ns, SITE_MMA + 9);
+                ok = wait_bar(slot_full(nk % SLOTS), (nk / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
                 if (!ok) break;
-                tc_fence_after();
-                qk(t, qb, nk % SLOTS);
-                umma_commit(s_full(t));
               }
               if (it > 0) {
-                ok = wait_bar(p_ready(t), (gi - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
-                // the first PV of a unit overwrites O_t: the previous unit's
-                // epilogue must have read it
-                if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+                ok = wait_bar(slot_full(nv % SLOTS), (nv / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
                 if (!ok) break;
-                tc_fence_after();
-                pv(t, nv % SLOTS, it > 1);
-                umma_commit(p_free(t));
-                if (it == u.nblk) umma_commit(o_full(t));
               }
-            }
-            if (!ok) break;
-            if (it < u.nblk) {
-              umma_commit(slot_empty(nk % SLOTS));
-              if (it == u.nblk - 1) umma_commit(q_empty(qb));  // the unit's last S products
-            }
-            if (it > 0) umma_commit(slot_empty(nv % SLOTS));
-          }
-          if (!ok) break;
-          n += 2 * u.nblk;
-          g += u.nblk;
-          L = fetch(k + 1);
-          ok = L != -2;
-          continue;
-        }
-        if (!s0_issued) {
-          const int sk = n % SLOTS;
-          ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
-          if (!ok) break;
-          tc_fence_after();
-          for (int t = 0; t < NQT; ++t) {
-            qk(t, qb, sk);
-            umma_commit(s_full(t));
-          }
-          umma_commit(slot_empty(sk));
-          if (u.nblk == 1) umma_commit(q_empty(qb));
-          ++n;
-        }
-        for (int it = 1; it < u.nblk && ok; ++it) {
-          const int sv = n % SLOTS, sk = (n + 1) % SLOTS;
-          ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
-          for (int t = 0; t < NQT && ok; ++t) {
-            ok = wait_bar(p_ready(t), (g + it - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
-            // the first PV of a unit overwrites O_t: the previous unit's
-            // epilogue must have read it
-            if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
-            if (!ok) break;
-            tc_fence_after();
-            pv(t, sv, it > 1);
-            if (t == 0) {
-              ok = wait_bar(slot_full(sk), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 4);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            qk(t, qb, sk);
-            umma_commit(s_full(t));
-          }
-          if (!ok) break;
-          if (it == u.nblk - 1) umma_commit(q_empty(qb));  // the unit's last S products
-          umma_commit(slot_empty(sv));
-          umma_commit(slot_empty(sk));
-          n += 2;
-        }
-        if (!ok) break;
-        // Last block: PV_t, then at once S_t of the next unit's first block
-        // (K in the slot after this unit's last V), so the softmax of tile t
-        // does not wait behind both tiles' last PV products at the boundary.
-        {
-          const int sv = n % SLOTS, skn = (n + 1) % SLOTS, qbn = (k + 1) & 1;
-          int Ln = -1;
-          Unit un{};
-          ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 5);
-          for (int t = 0; t < NQT && ok; ++t) {
-            ok = wait_bar(p_ready(t), (g + u.nblk - 1) & 1, ab, p.wait_ns, SITE_MMA + 6);
-            if (ok && u.nblk == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
-            if (!ok) break;
-            tc_fence_after();
-            pv(t, sv, u.nblk > 1);
-            umma_commit(o_full(t));
-            if (t == 0) {
-              Ln = fetch(k + 1);
-              ok = Ln != -2;
-              if (ok && Ln >= 0) {
-                un = unit_of<MODE>(p, Ln);
-                ok = wait_bar(q_full(qbn), ((k + 1) >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
-                if (ok) ok = wait_bar(slot_full(skn), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
-                if (ok) tc_fence_after();
+              for (int t = 0; t < NQT && ok; ++t) {
+                if (it < u.nblk) {
+                  if (gi > 0) ok = wait_bar(s_read(t), (gi - 1) & 1, ab, p.wait_ns, SITE_MMA + 9);
+                  if (!ok) break;
+                  tc_fence_after();
+                  qk(t, qb, nk % SLOTS);
+                  umma_commit(s_full(t));
+                }
+                if (it > 0) {
+                  ok = wait_bar(p_ready(t), (gi - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
+                  // the first PV of a unit overwrites O_t: the previous unit's
+                  // epilogue must have read it
+                  if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+                  if (!ok) break;
+                  tc_fence_after();
+                  pv(t, nv % SLOTS, it > 1);
+                  umma_commit(p_free(t));
+                  if (it == u.nblk) umma_commit(o_full(t));
+                }
               }
               if (!ok) break;
+              if (it < u.nblk) {
+                umma_commit(slot_empty(nk % SLOTS));
+                if (it == u.nblk - 1) umma_commit(q_empty(qb));  // the unit's last S products
+              }
+              if (it > 0) umma_commit(slot_empty(nv % SLOTS));
             }
-            if (Ln >= 0) {
-              qk(t, qbn, skn);
+            if (!ok) break;
+            n += 2 * u.nblk;
+            g += u.nblk;
+            continue;
+          }
+          {
+            const int sk = n % SLOTS;
+            ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
+            if (!ok) break;
+            tc_fence_after();
+            for (int t = 0; t < NQT; ++t) {
+              qk(t, qb, sk);
               umma_commit(s_full(t));
             }
-          }
-          if (!ok) break;
-          umma_commit(slot_empty(sv));
-          ++n;
-          if (Ln >= 0) {
-            umma_commit(slot_empty(skn));
-            if (un.nblk == 1) umma_commit(q_empty(qbn));
+            umma_commit(slot_empty(sk));
+            if (u.nblk == 1) umma_commit(q_empty(qb));
             ++n;
           }
-          L = Ln;
-          s0_issued = true;
+          for (int it = 1; it < u.nblk && ok; ++it) {
+            const int sv = n % SLOTS, sk = (n + 1) % SLOTS;
+            ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
+            for (int t = 0; t < NQT && ok; ++t) {
+              ok = wait_bar(p_ready(t), (g + it - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
+              // the first PV of a unit overwrites O_t: the previous unit's
+              // epilogue must have read it
+              if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+              if (!ok) break;
+              tc_fence_after();
+              pv(t, sv, it > 1);
+              if (t == 0) {
+                ok = wait_bar(slot_full(sk), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 4);
+                if (!ok) break;
+                tc_fence_after();
+              }
+              qk(t, qb, sk);
+              umma_commit(s_full(t));
+            }
+            if (!ok) break;
+            if (it == u.nblk - 1) umma_commit(q_empty(qb));  // the unit's last S products
+            umma_commit(slot_empty(sv));
+            umma_commit(slot_empty(sk));
+            n += 2;
+          }
+          if (!ok) break;
+          {
+            const int sv = n % SLOTS;
+            ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 5);
+            for (int t = 0; t < NQT && ok; ++t) {
+              ok = wait_bar(p_ready(t), (g + u.nblk - 1) & 1, ab, p.wait_ns, SITE_MMA + 6);
+              if (ok && u.nblk == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+              if (!ok) break;
+              tc_fence_after();
+              pv(t, sv, u.nblk > 1);
+              umma_commit(o_full(t));
+            }
+            if (ok) umma_commit(slot_empty(sv));
+            ++n;
+          }
+          g += u.nblk;
         }
-        g += u.nblk;
+      } else {
+        // Static schedule, P over S: the last block of a unit issues PV_t
+        // and at once S_t of the next unit's first block (K in the slot after
+        // this unit's last V), so the softmax of tile t does not wait behind
+        // both tiles' last PV products at the boundary.  The loader runs a
+        // whole unit ahead here; with the shared counter (short units, the
+        // next unit known late) the plain order above measured faster.
+        auto fetch = [&](int k) -> int {
+          const int L = unit_index(k);
+          return L >= p.num_units ? -1 : L;
+        };
+        int n = 0, g = 0;  // KV slots, blocks
+        bool ok = true;
+        // this unit's first S products went out with the previous unit's last
+        // PV products (every unit but the first)
+        bool s0_issued = false;
+        int L = fetch(0);
+        for (int k = 0; ok && L >= 0; ++k) {
+          const Unit u = unit_of<MODE>(p, L);
+          const int qb = k & 1;
+          if (!s0_issued) {
+            ok = wait_bar(q_full(qb), (k >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
+            if (!ok) break;
+            const int sk = n % SLOTS;
+            ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
+            if (!ok) break;
+            tc_fence_after();
+            for (int t = 0; t < NQT; ++t) {
+              qk(t, qb, sk);
+              umma_commit(s_full(t));
+            }
+            umma_commit(slot_empty(sk));
+            if (u.nblk == 1) umma_commit(q_empty(qb));
+            ++n;
+          }
+          for (int it = 1; it < u.nblk && ok; ++it) {
+            const int sv = n % SLOTS, sk = (n + 1) % SLOTS;
+            ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
+            for (int t = 0; t < NQT && ok; ++t) {
+              ok = wait_bar(p_ready(t), (g + it - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
+              // the first PV of a unit overwrites O_t: the previous unit's
+              // epilogue must have read it
+              if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+              if (!ok) break;
+              tc_fence_after();
+              pv(t, sv, it > 1);
+              if (t == 0) {
+                ok = wait_bar(slot_full(sk), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 4);
+                if (!ok) break;
+                tc_fence_after();
+              }
+              qk(t, qb, sk);
+              umma_commit(s_full(t));
+            }
+            if (!ok) break;
+            if (it == u.nblk - 1) umma_commit(q_empty(qb));  // the unit's last S products
+            umma_commit(slot_empty(sv));
+            umma_commit(slot_empty(sk));
+            n += 2;
+          }
+          if (!ok) break;
+          {  // last block, with the next unit's first S products
+            const int sv = n % SLOTS, skn = (n + 1) % SLOTS, qbn = (k + 1) & 1;
+            int Ln = -1;
+            Unit un{};
+            ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 5);
+            for (int t = 0; t < NQT && ok; ++t) {
+              ok = wait_bar(p_ready(t), (g + u.nblk - 1) & 1, ab, p.wait_ns, SITE_MMA + 6);
+              if (ok && u.nblk == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+              if (!ok) break;
+              tc_fence_after();
+              pv(t, sv, u.nblk > 1);
+              umma_commit(o_full(t));
+              if (t == 0) {
+                Ln = fetch(k + 1);
+                if (Ln >= 0) {
+                  un = unit_of<MODE>(p, Ln);
+                  ok = wait_bar(q_full(qbn), ((k + 1) >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
+                  if (ok) ok = wait_bar(slot_full(skn), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
+                  if (ok) tc_fence_after();
+                }
+                if (!ok) break;
+              }
+              if (Ln >= 0) {
+                qk(t, qbn, skn);
+                umma_commit(s_full(t));
+              }
+            }
+            if (!ok) break;
+            umma_commit(slot_empty(sv));
+            ++n;
+            if (Ln >= 0) {
+              umma_commit(slot_empty(skn));
+              if (un.nblk == 1) umma_commit(q_empty(qbn));
+              ++n;
+            }
+            L = Ln;
+            s0_issued = true;
+          }
+          g += u.nblk;
+        }
       }
       // Drain: wait until every MMA issued above has completed.
       umma_commit(drain_bar);
