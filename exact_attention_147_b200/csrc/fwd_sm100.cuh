@@ -9,11 +9,13 @@
 // single long head already fills the GPU and one unit's loads and first
 // products overlap the previous unit's epilogue.
 //
-// Inside a CTA (10 warps):
+// Inside a CTA (16 warps, four warpgroups):
 //   warps 0-3   softmax for query tile 0 (thread = one query row)
 //   warps 4-7   softmax for query tile 1
-//   warp  8     TMA producer: Q once, then K_j, V_j into a ring of slots
-//   warp  9     MMA issuer: S_t = Q_t K_j^T and O_t += P_t V_j (tcgen05)
+//   warps 8-11  epilogue: O_t / l out of TMEM, bf16 rows and LSE to HBM
+//   warp  12    TMA producer: Q once per unit, then K_j, V_j into a ring of slots
+//   warp  13    MMA issuer: S_t = Q_t K_j^T and O_t += P_t V_j (tcgen05)
+//   warps 14-15 idle (they complete the fourth warpgroup for setmaxnreg)
 // The Q tiles stay resident in shared memory and K/V tiles stream through a
 // multi-slot TMA + mbarrier ring ("FlashAttention v2" article, §3.1-§3.2:
 // Q kept on chip, K/V prefetched while the current block is computed).
