@@ -904,8 +904,9 @@ __global__ void __launch_bounds__(192, 1) fa2_bwd_dq_sm100_kernel(const __grid_c
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // the query blocks of one head are launched together (they share its K
-  // and V in L2)
-  const int qb = int(blockIdx.x % p.nblocks);
+  // and V in L2), the last one first: under a causal mask it visits the most
+  // key blocks, so the grid ends on short blocks rather than long ones
+  const int qb = p.nblocks - 1 - int(blockIdx.x % p.nblocks);
   const int hb = int(blockIdx.x / p.nblocks);
   const int h = hb % p.H, b = hb / p.H;
   const SeqView sv = PACKED ? seq_view(p.cu_seqlens, b, p.N, p.total) : SeqView{b, 0, p.N};
