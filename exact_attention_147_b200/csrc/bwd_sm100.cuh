@@ -279,12 +279,14 @@ __device__ __forceinline__ void st_global_row32(__nv_bfloat16* base, const Strid
 // acc_empty), and g, the query blocks it has processed (the Q / dO rings
 // and the per-block barriers).
 // ---------------------------------------------------------------------------
-template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT, int MODE>
+// DSCHED: padded calls whose items differ in cost (a causal mask over many
+// key blocks) also take their items from the shared counter.
+template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT, int MODE, bool DSCHED = false>
 __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<HD>;
   constexpr bool PACKED = MODE == kLayoutPacked;
   constexpr bool SPARSE = MODE == kLayoutSparse;
-  constexpr bool DYN = PACKED || SPARSE;  // items taken from the shared counter
+  constexpr bool DYN = PACKED || SPARSE || DSCHED;  // items taken from the shared counter
   using namespace bwd_detail;
   constexpr int QS = C::Q_STAGES, DS = C::DO_STAGES;
   constexpr int NCH = HD / 64;

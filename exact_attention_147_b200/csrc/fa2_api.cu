@@ -314,6 +314,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
                             const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
                             int dev, cudaStream_t st) {
   static std::atomic<uint64_t> mask_dkdv{0}, mask_dkdv_nodq{0}, mask_dq{0};
+  static std::atomic<uint64_t> mask_dkdv_dyn{0}, mask_dkdv_nodq_dyn{0};
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
   const MapShape ms = map_shape(a);
@@ -361,7 +362,21 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
     FA2_TRY(current_device(&dev2, &di));
   }
   const unsigned grid1 = std::min<unsigned>(grid, unsigned(std::max(di.sm_count, 1)));
-  if (MODE != kLayoutPadded) FA2_TRY(sched_counters(dev, &p.sched));
+  // Under a causal mask (right window 0) key block j of a head has nq - j
+  // query blocks.  With many key blocks the static snake leaves some CTAs far
+  // behind the rest (25 % over the mean at N = 16384, simulated), so such
+  // calls take their items from the shared counter in the same head-major
+  // order.  Measured (d = 128, B N = 16384): the counter wins from 128 key
+  // blocks on (N = 16384: +9 %; d = 64: +5 %; window (4096, 0) at N = 32768:
+  // +1 %) and loses below (N = 4096: -3 %, N = 8192: -5 %).
+  constexpr bool CAN_DYN = MODE == kLayoutPadded;
+  const bool dyn = CAN_DYN && a.wr == 0 && p.nblocks >= 128;
+  if (MODE != kLayoutPadded || dyn) FA2_TRY(sched_counters(dev, &p.sched));
+  using K1 = void (*)(BwdParams);
+  const K1 k1_dq = dyn ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE, CAN_DYN>
+                       : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE>;
+  const K1 k1_nodq = dyn ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, MODE, CAN_DYN>
+                         : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, MODE>;
   constexpr int smem1 = BwdCfg<HD>::SMEM_BYTES;
   // Kernel 1 re-balances registers between its warpgroups; the shares add up
   // to 512 threads x REGS_AT_LAUNCH, so the compiled kernel must launch with
@@ -369,9 +384,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   // forever.  Refuse to launch otherwise.
   {
     cudaFuncAttributes fa;
-    auto k1c = deterministic ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, MODE>
-                             : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE>;
-    if (cudaFuncGetAttributes(&fa, k1c) != cudaSuccess) return FA2_ERR_CUDA;
+    if (cudaFuncGetAttributes(&fa, deterministic ? k1_nodq : k1_dq) != cudaSuccess) return FA2_ERR_CUDA;
     if (fa.numRegs < BwdCfg<HD>::REGS_AT_LAUNCH) return FA2_ERR_UNSUPPORTED;
   }
   if (!deterministic) {
@@ -379,9 +392,8 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
     const unsigned zgrid = unsigned(std::min<long long>((n4 + 255) / 256, 148 * 16));
     zero_f32x4_kernel<<<zgrid, 256, 0, st>>>(reinterpret_cast<float4*>(a.dq_accum), n4);
     FA2_TRY(launched(1));
-    auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE>;
-    FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv));
-    k1<<<grid1, BwdCfg<HD>::THREADS, smem1, st>>>(p);
+    FA2_TRY(ensure_smem(k1_dq, smem1, dev, dyn ? mask_dkdv_dyn : mask_dkdv));
+    k1_dq<<<grid1, BwdCfg<HD>::THREADS, smem1, st>>>(p);
     FA2_TRY(launched(1));
     AttnArgs c = a;  // the accumulator is [bt * H, rows, d] in both layouts
     c.B = ms.bt;
@@ -392,9 +404,8 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
     dq_convert_kernel<HD><<<unsigned((rows + per_block - 1) / per_block), 256, 0, st>>>(c);
     return launched(1);
   }
-  auto k1 = fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, MODE>;
-  FA2_TRY(ensure_smem(k1, smem1, dev, mask_dkdv_nodq));
-  k1<<<grid1, BwdCfg<HD>::THREADS, smem1, st>>>(p);
+  FA2_TRY(ensure_smem(k1_nodq, smem1, dev, dyn ? mask_dkdv_nodq_dyn : mask_dkdv_nodq));
+  k1_nodq<<<grid1, BwdCfg<HD>::THREADS, smem1, st>>>(p);
   FA2_TRY(launched(1));
   auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI, DROPOUT, MODE>;
   constexpr int smem2 = DqCfg<HD>::SMEM_BYTES;

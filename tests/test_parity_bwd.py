@@ -89,6 +89,13 @@ def test_sweep_sampled(n, d):
     compare_heads(w, [(w.B - 1, w.H - 1)])
 
 
+def test_causal_long_sampled():
+    # 128 key blocks under a causal mask: the dK/dV kernel takes its items
+    # from the shared counter
+    w = W.sweep(16384, 128, causal=True)
+    compare_heads(w, [(0, w.H - 1)])
+
+
 def test_long_local_sampled():
     w = W.long_local()
     compare_heads(w, [(0, 31)])
