@@ -221,15 +221,17 @@ __device__ __forceinline__ int next_qblock(const BwdParams& p, const BItem& it, 
   return MODE == kLayoutSparse ? next_kept(it.mcol, p.nb, qb, it.qb_last) : qb + 1;
 }
 
-// Static schedule of kernel 1 (padded calls): the k-th item of CTA c in a
-// persistent grid of G CTAs, a snake over the item order.
+// Static schedule of kernel 1 (padded calls, except causal ones with 128 or
+// more key blocks): the k-th item of CTA c in a persistent grid of G CTAs, a
+// snake over the item order.
 __device__ __forceinline__ int bwd_item_index(int k) {
   const int G = int(gridDim.x), c = int(blockIdx.x);
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-// Packed / block-sparse calls: items taken from a shared counter as CTAs
-// become free (their cost follows the lengths or the mask).  Next non-empty
+// Packed and block-sparse calls, and long causal padded calls: items taken
+// from a shared counter as CTAs become free (their cost follows the lengths,
+// the mask or the key block's place under the causal mask).  Next non-empty
 // item, or -1.  Only the producer thread calls this.
 template <int MODE>
 __device__ __forceinline__ int fetch_item(const BwdParams& p) {
