@@ -34,8 +34,13 @@
  *    16-byte aligned.  lse and D are dense fp32 [B, H, N].
  *  - All pointers are DEVICE pointers, owned by the caller; the library
  *    allocates no device memory and keeps no state between calls except a
- *    small cache of device properties and the device status word read by
- *    fa2_device_status().
+ *    small cache of device properties, the device status word read by
+ *    fa2_device_status(), and a table of 64 work counters.  Calls whose work
+ *    items differ in cost (the *_varlen and *_blocksparse calls, and
+ *    backward calls with a causal mask over 128 or more key blocks) take
+ *    their items from one of these counters, in turn, and the last CTA of
+ *    the call resets it.  At most 64 such calls may therefore run at the
+ *    same time on one device (on different streams).
  *  - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
  *    default stream); nothing is synchronised.
  *  - Every argument is checked before anything is launched.  An invalid
