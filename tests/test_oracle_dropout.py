@@ -20,6 +20,35 @@ from oracle import philox
 RNG = np.random.default_rng(777)
 
 
+# Known-answer vectors of Philox4x32-10 published with the generator's
+# reference implementation (Random123, the "kat_vectors" file that
+# accompanies Salmon et al., SC 2011): (counter c0..c3, key k0, k1) ->
+# output words.  A wrong multiplier, Weyl constant, round count or word
+# order changes every one of them.
+PHILOX_KAT = [
+    ((0x00000000, 0x00000000, 0x00000000, 0x00000000), (0x00000000, 0x00000000),
+     (0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8)),
+    ((0xFFFFFFFF, 0xFFFFFFFF, 0xFFFFFFFF, 0xFFFFFFFF), (0xFFFFFFFF, 0xFFFFFFFF),
+     (0x408F276D, 0x41C83B0E, 0xA20BC7C6, 0x6D5451FD)),
+    ((0x243F6A88, 0x85A308D3, 0x13198A2E, 0x03707344), (0xA4093822, 0x299F31D0),
+     (0xD16CFE09, 0x94FDCCEB, 0x5001E420, 0x24126EA1)),
+]
+
+
+@pytest.mark.parametrize("ctr,key,expect", PHILOX_KAT)
+def test_philox_known_answers(ctr, key, expect):
+    got = philox.philox4x32_10(*[np.uint32(c) for c in ctr], *key)
+    assert tuple(int(x) for x in got) == expect
+
+
+def test_philox_known_answers_vectorised():
+    # the same vectors through the broadcasting path the mask generator uses
+    c = np.array([v[0] for v in PHILOX_KAT], dtype=np.uint32).T
+    for (ctr, key, expect), col in zip(PHILOX_KAT, range(c.shape[1])):
+        got = philox.philox4x32_10(c[0], c[1], c[2], c[3], *key)
+        assert tuple(int(w[col]) for w in got) == expect
+
+
 def test_philox_is_a_deterministic_function_of_counter_and_key():
     c = RNG.integers(0, 2**32, size=(4, 1000), dtype=np.uint64).astype(np.uint32)
     a = philox.philox4x32_10(*c, 123, 456)

@@ -1,11 +1,15 @@
 """Dropout parity: libfa2's dropout mask and gradients against the oracle.
 
 The mask itself is compared bit for bit: with q = 0 every visible key gets
-the same probability, so a one-hot value row makes each output element
-count the kept keys that land on it (forward), and a one-hot dO row does the
-same for dV (backward key-row kernel).  Outputs and gradients are then
-compared with the fp64 oracle, which draws the same mask with its own
-Philox4x32-10.
+the same probability 1/N, so when value row j is the unit vector e_(j mod d)
+for the keys of one half of the sequence and zero for the other half, output
+element (i, c) is keep(i, j) / N times the keep scale for the single key j
+of that half with j mod d = c (forward); one-hot dO rows over one half of
+the queries do the same for dV (backward key-row kernel).  Each half is its
+own call, so every element of the mask is read on its own.  Outputs and
+gradients are then compared with the fp64 oracle, which draws the same mask
+with its own Philox4x32-10 (pinned to the generator's published
+known-answer vectors in tests/test_oracle_dropout.py).
 """
 
 import numpy as np
@@ -21,9 +25,12 @@ from tests.helpers import check_fwd, check_grad, f64
 pytestmark = pytest.mark.gpu
 
 
-def onehot_rows(n, d, dtype):
+def onehot_half(n, d, half, dtype):
+    """[n, d]: row j is e_(j mod d) for the rows of half `half` (d rows each),
+    zero elsewhere."""
     v = torch.zeros(n, d)
-    v[torch.arange(n), torch.arange(n) % d] = 1.0
+    rows = torch.arange(half * d, (half + 1) * d)
+    v[rows, rows % d] = 1.0
     return v.to(dtype)
 
 
@@ -34,26 +41,28 @@ def test_mask_bits_forward_and_backward(dtype, p, seed):
     q = torch.zeros(B, N, H, d, dtype=dtype, device="cuda")
     g = torch.Generator().manual_seed(3)
     k = torch.randn(B, N, H, d, generator=g).to(dtype).cuda()
-    base = onehot_rows(N, d, dtype)                      # key j -> column j mod d
-    v = base[None, :, None, :].expand(B, N, H, d).contiguous().cuda()
-    out, lse = F.fwd(q, k, v, dropout_p=p, dropout_seed=seed)
-    do = base[None, :, None, :].expand(B, N, H, d).contiguous().cuda()  # query i -> column i mod d
-    D = F.bwd_preprocess(out, do)
-    dq, dk, dv = F.bwd(do, q, k, v, lse, D, dropout_p=p, dropout_seed=seed)
-    torch.cuda.synchronize()
-    assert F.device_status() == 0
     ks = philox.keep_scale(p)
-    for b in range(B):
-        for h in range(H):
-            keep = philox.keep_mask(b, h, np.arange(N), N, p, seed).astype(np.float64)
-            # forward: O[i, c] = ks / N * (# kept keys j with j mod d == c)
-            cnt_f = keep.reshape(N, N // d, d).sum(axis=1)
-            got_f = np.rint(f64(out[b, :, h]) * N / ks)
-            assert np.array_equal(got_f, cnt_f), f"forward mask mismatch b={b} h={h}"
-            # backward: dV[j, c] = ks / N * (# kept queries i with i mod d == c)
-            cnt_b = keep.T.reshape(N, N // d, d).sum(axis=1)
-            got_b = np.rint(f64(dv[b, :, h]) * N / ks)
-            assert np.array_equal(got_b, cnt_b), f"backward mask mismatch b={b} h={h}"
+    keep = {(b, h): philox.keep_mask(b, h, np.arange(N), N, p, seed).astype(np.float64)
+            for b in range(B) for h in range(H)}
+    for half in range(N // d):
+        base = onehot_half(N, d, half, dtype)
+        sl = slice(half * d, (half + 1) * d)
+        # value rows of keys in this half only: O[i, c] = ks / N * keep[i, half*d + c]
+        v = base[None, :, None, :].expand(B, N, H, d).contiguous().cuda()
+        out, lse = F.fwd(q, k, v, dropout_p=p, dropout_seed=seed)
+        # dO rows of queries in this half only: dV[j, c] = ks / N * keep[half*d + c, j]
+        do = base[None, :, None, :].expand(B, N, H, d).contiguous().cuda()
+        D = F.bwd_preprocess(out, do)
+        dq, dk, dv = F.bwd(do, q, k, v, lse, D, dropout_p=p, dropout_seed=seed)
+        torch.cuda.synchronize()
+        assert F.device_status() == 0
+        for b in range(B):
+            for h in range(H):
+                m = keep[(b, h)]
+                got_f = np.rint(f64(out[b, :, h]) * N / ks)
+                assert np.array_equal(got_f, m[:, sl]), f"forward mask b={b} h={h} half={half}"
+                got_b = np.rint(f64(dv[b, :, h]) * N / ks)
+                assert np.array_equal(got_b, m[sl, :].T), f"backward mask b={b} h={h} half={half}"
 
 
 CASES = [
