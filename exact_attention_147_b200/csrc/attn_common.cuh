@@ -92,6 +92,19 @@ __device__ __forceinline__ SeqView seq_view(const int* cu, int b, int N, int tot
   return s;
 }
 
+// Counter-scheduled calls (work items taken from a shared counter pair
+// {next item, finished CTAs}): each CTA calls this once, from one thread,
+// when it takes no further item -- including a CTA that stops before taking
+// any -- and the call's last CTA returns the pair to zero.
+__device__ __forceinline__ void sched_cta_done(unsigned int* sched) {
+  __threadfence();
+  if (atomicAdd(sched + 1, 1u) == gridDim.x - 1) {
+    sched[0] = 0u;
+    sched[1] = 0u;
+    __threadfence();
+  }
+}
+
 // Element pointer of row i, head h of a [B, N, H, d] / [total, H, d] tensor.
 template <typename T, typename P>
 __device__ __forceinline__ T* row_ptr(P* base, const Strides& s, const SeqView& v, int i, int h) {

@@ -69,6 +69,8 @@ struct BwdParams {
   DropoutParams drop;                    // used by the DROPOUT instantiations
   int num_items;                         // key blocks x heads x batch (kernel 1 work items)
   unsigned int* sched;                   // packed / block-sparse kernel 1: {next item, finished CTAs}
+  uint32_t* dq_chain;                    // ordered dQ: [B*H, nblocks, 4] counters (zero at launch)
+  int test_skip;                         // test switch, 0 in normal use: see kernel 1's ds_ready arrive
 };
 
 template <int HD>
@@ -176,14 +178,15 @@ struct BItem {
   bool empty;
 };
 
-template <int MODE>
+template <int MODE, bool ORDER = false>
 __device__ __forceinline__ BItem item_of(const BwdParams& p, int I) {
   BItem it;
   // Key blocks of one head together, masked or not: they share the head's
   // Q and dO in L2.  (Ordering all heads' block 0 first, the longest-first
   // order for causal masks, ran 148 heads at once and lost 20 % to L2
-  // misses.)
-  it.kb = I % p.nblocks;
+  // misses.)  The ordered-dQ kernel takes a head's key blocks last first
+  // (see its dQ drain).
+  it.kb = ORDER ? p.nblocks - 1 - I % p.nblocks : I % p.nblocks;
   const int hb = I / p.nblocks;
   it.h = hb % p.H;
   it.b = hb / p.H;
@@ -233,12 +236,12 @@ __device__ __forceinline__ int bwd_item_index(int k) {
 // from a shared counter as CTAs become free (their cost follows the lengths,
 // the mask or the key block's place under the causal mask).  Next non-empty
 // item, or -1.  Only the producer thread calls this.
-template <int MODE>
+template <int MODE, bool ORDER = false>
 __device__ __forceinline__ int fetch_item(const BwdParams& p) {
   for (;;) {
     const int I = int(atomicAdd(p.sched, 1u));
     if (I >= p.num_items) return -1;
-    if (!item_of<MODE>(p, I).empty) return I;
+    if (!item_of<MODE, ORDER>(p, I).empty) return I;
   }
 }
 
@@ -283,8 +286,12 @@ __device__ __forceinline__ void st_global_row32(__nv_bfloat16* base, const Strid
 // ---------------------------------------------------------------------------
 // DSCHED: padded calls whose items differ in cost (a causal mask over many
 // key blocks) also take their items from the shared counter.
-template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT, int MODE, bool DSCHED = false>
+// ORDER: deterministic dQ under a causal mask (padded layout, with DSCHED):
+// the partial dQ tiles of a query block are added in a fixed order (see the
+// dQ drain), so dq is bitwise repeatable without a second pass.
+template <int HD, bool ALIBI, bool WITH_DQ, bool DROPOUT, int MODE, bool DSCHED = false, bool ORDER = false>
 __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid_constant__ BwdParams p) {
+  static_assert(!ORDER || (WITH_DQ && DSCHED && MODE == kLayoutPadded), "ordered dQ: padded, counter-scheduled");
   using C = BwdCfg<HD>;
   constexpr bool PACKED = MODE == kLayoutPacked;
   constexpr bool SPARSE = MODE == kLayoutSparse;
@@ -296,7 +303,10 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {  // 128-byte-swizzled tiles need 1 KB alignment
-    if (threadIdx.x == 0) atomicCAS(&g_fa2_device_status, 0, SITE_SMEM_ALIGN);
+    if (threadIdx.x == 0) {
+      atomicCAS(&g_fa2_device_status, 0, SITE_SMEM_ALIGN);
+      if (DYN) sched_cta_done(p.sched);  // takes no item, but must still count as finished
+    }
     return;
   }
   uint8_t* smem = smem_raw;
@@ -373,7 +383,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         I = -1;
         return true;
       }
-      if (!item_of<MODE>(p, I).empty) return true;
+      if (!item_of<MODE, ORDER>(p, I).empty) return true;
     }
   };
 
@@ -383,7 +393,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       // ---------------------------------------------------------- producer
       int issued_q = 0, issued_do = 0, issued_kv = 0, jn = 0, g = 0, k = 0;
       bool ok = true;
-      int I = DYN ? (lane == 0 ? fetch_item<MODE>(p) : 0) : -1;
+      int I = DYN ? (lane == 0 ? fetch_item<MODE, ORDER>(p) : 0) : -1;
       if (DYN) I = __shfl_sync(0xffffffffu, I, 0);
       for (;;) {
         if (DYN) {  // publish the item (or the end mark -1) to the other roles
@@ -400,11 +410,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         } else {
           for (;;) {  // the static schedule, skipping empty items
             I = bwd_item_index(k++);
-            if (I >= p.num_items || !item_of<MODE>(p, I).empty) break;
+            if (I >= p.num_items || !item_of<MODE, ORDER>(p, I).empty) break;
           }
           if (I >= p.num_items) break;
         }
-        const BItem itm = item_of<MODE>(p, I);
+        const BItem itm = item_of<MODE, ORDER>(p, I);
         int I_next = 0;
         // K and V of this item once the previous item's products have read them
         ok = wait_bar(kv_empty, (jn & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 2);
@@ -418,8 +428,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           }
         }
         ++issued_kv;
-        // the next item's index: the atomic is in flight while this item loads
-        if (DYN && lane == 0) I_next = fetch_item<MODE>(p);
+        // the next item's index: the atomic is in flight while this item
+        // loads.  (The ordered dQ claims its next item only once this item's
+        // loads are out, about one query block before it can start: claims
+        // must start in the order they were made, see the dQ drain.)
+        if (DYN && !ORDER && lane == 0) I_next = fetch_item<MODE, ORDER>(p);
         int qb = itm.qb_first;
         for (int it = 0; it < itm.nq && ok; ++it, qb = next_qblock<MODE>(p, itm, qb)) {
           const int gi = g + it;
@@ -471,19 +484,13 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           ++issued_do;
         }
         if (!ok) break;
+        if (ORDER && lane == 0) I_next = fetch_item<MODE, ORDER>(p);
         g += itm.nq;
         ++jn;
         if (DYN) I = __shfl_sync(0xffffffffu, I_next, 0);
       }
-      if (DYN && lane == 0) {
-        // The last CTA to finish taking items returns the counters to zero.
-        __threadfence();
-        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
-          p.sched[0] = 0u;
-          p.sched[1] = 0u;
-          __threadfence();
-        }
-      }
+      // The last CTA to finish taking items returns the counters to zero.
+      if (DYN && lane == 0) sched_cta_done(p.sched);
       if (lane == 0) {  // every copy issued must land before the CTA exits
         if (issued_kv > 0) drain_wait(kv_full, (issued_kv - 1) & 1, p.wait_ns);
         for (int q = max(0, issued_q - QS); q < issued_q; ++q)
@@ -555,7 +562,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         I = __shfl_sync(0xffffffffu, I, 0);
         if (!ok || I < 0) break;
-        const BItem itm = item_of<MODE>(p, I);
+        const BItem itm = item_of<MODE, ORDER>(p, I);
         const int nq = itm.nq;
         if (lane == 0) {
           ok = wait_bar(kv_full, jn & 1, ab, p.wait_ns, SITE_BMMA + 0);
@@ -615,7 +622,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       int I;
       ok = next_item(k, I, true, SITE_BCOMP + 3);
       if (!ok || I < 0) break;
-      const BItem itm = item_of<MODE>(p, I);
+      const BItem itm = item_of<MODE, ORDER>(p, I);
       const int h = itm.h, b = itm.b;
       const int j = itm.k0 + r;
       int lo_q = p.wr >= 0 ? max(0, j - p.wr) : 0;
@@ -755,7 +762,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         tmem_st_wait();
         if (WITH_DQ) fence_proxy_async_smem();
         tc_fence_before();
-        bar_arrive(ds_ready);
+        // Test switch (off in normal use): in the CTA that takes item 0 (its
+        // first item, whichever schedule), compute warpgroup 0 withholds its
+        // arrive on the first query block, so the MMA warp's bounded wait
+        // for dS runs out and every role of that CTA winds down.
+        if (!(p.test_skip && I == 0 && it == 0 && wg == 0)) bar_arrive(ds_ready);
       }
       if (!ok) break;
       // -------------------------------------------------------- item epilogue
@@ -805,11 +816,25 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       const int wq = warp % 4;
       int g = 0, k = 0;
       bool ok = true;
+      // Ordered dQ: the box (this warp's 32 rows of a query block) whose adds
+      // were issued last and whose counter is still to be raised.
+      long long pend_box = -1;
+      uint32_t pend_val = 0;
+      auto chain_release = [&]() {
+        if (ORDER && pend_box >= 0) {
+          if (lane == 0) {
+            bulk_wait_all();              // this warp's adds into the box are complete
+            fence_proxy_async_global();
+            st_release_gpu(p.dq_chain + pend_box, pend_val);
+          }
+          pend_box = -1;
+        }
+      };
       for (;;) {
         int I;
         ok = next_item(k, I, true, SITE_BRED + 1);
         if (!ok || I < 0) break;
-        const BItem itm = item_of<MODE>(p, I);
+        const BItem itm = item_of<MODE, ORDER>(p, I);
         const int bh = itm.bt * p.H + itm.h;
         int qb = itm.qb_first;
         for (int it = 0; it < itm.nq; ++it, qb = next_qblock<MODE>(p, itm, qb)) {
@@ -849,11 +874,36 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           tmem_ld_wait();
           tc_fence_before();
           bar_arrive(dq_free);   // TMEM columns may now take the next dP^T
+          if (ORDER) {
+            // Deterministic dQ under a causal mask: every box takes the key
+            // blocks' partial sums in descending key-block order.  Key block
+            // kb reaches query block qb after qb - kb steps of its own walk,
+            // which is its rank in that order, and the key blocks of a head
+            // are taken last first, so a partial sum arrives about when its
+            // turn comes and only ever waits for items taken earlier (no
+            // wait can close a cycle).  The box's counter holds how many sums
+            // it has received: wait for our rank, add, and raise the counter
+            // once the adds are complete (at the next box, or at the end of
+            // the item).
+            chain_release();
+            const long long box = ((long long)bh * p.nblocks + qb) * 4 + wq;
+            const uint32_t rank = uint32_t(qb - itm.kb);
+            bool turn = true;
+            if (lane == 0) {
+              turn = wait_counter_eq(p.dq_chain + box, rank, ab, p.wait_ns, SITE_BRED + 3);
+              if (turn) fence_proxy_async_global();
+            }
+            ok = __shfl_sync(0xffffffffu, turn ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            pend_box = box;
+            pend_val = rank + 1u;
+          }
 #pragma unroll
           for (int c = 0; c < NC; ++c) stage(u[c], c);
         }
         if (!ok) break;
         g += itm.nq;
+        chain_release();
       }
       if (lane == 0) bulk_wait_all();
     } else if (DYN) {

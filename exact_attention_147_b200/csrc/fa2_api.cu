@@ -29,6 +29,7 @@ using namespace fa2;
 namespace {
 
 std::atomic<unsigned long long> g_wait_ns{1000ull * 1000ull * 1000ull};
+std::atomic<int> g_test_skip{0};  // fa2_test_skip_arrive: 0 off, 1 forward, 2 backward
 std::atomic<uint64_t> g_launches{0};
 
 constexpr int kMaxDevices = 64;
@@ -85,10 +86,23 @@ DropoutParams make_dropout(float dropout_p, unsigned long long seed) {
   } while (0)
 
 // ----------------------------------------------------------------- device
+// Device objects of the library that host code needs the address of: the
+// work counters of the counter-scheduled calls and the scratch of
+// fa2_bwd_noalloc.  In host code these names are only stand-ins for the
+// device objects; their device addresses come from cudaGetSymbolAddress,
+// looked up once per device, with that device current, the first time any
+// entry point reaches the device, so that no later call (one made during
+// stream capture, say) has to.
+constexpr int kSchedSlots = 64;
+static __device__ unsigned int g_fa2_sched[2 * kSchedSlots];
+static __device__ __align__(256) float g_fa2_noalloc_dq[FA2_NOALLOC_MAX_DQ_FLOATS];
+
 struct DeviceInfo {
   int sm_major = -1;
   int sm_minor = -1;
   int sm_count = 0;
+  unsigned int* sched = nullptr;  // device address of g_fa2_sched
+  float* noalloc_dq = nullptr;    // device address of g_fa2_noalloc_dq
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -99,12 +113,18 @@ fa2_status current_device(int* dev, DeviceInfo* info) {
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DeviceInfo& di = g_dev[*dev];
   if (di.sm_major < 0) {
-    if (cudaDeviceGetAttribute(&di.sm_major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&di.sm_minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess) {
-      di.sm_major = -1;
+    DeviceInfo n;
+    void* sched = nullptr;
+    void* scratch = nullptr;
+    if (cudaDeviceGetAttribute(&n.sm_major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n.sm_minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n.sm_count, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess ||
+        cudaGetSymbolAddress(&sched, g_fa2_sched) != cudaSuccess || sched == nullptr ||
+        cudaGetSymbolAddress(&scratch, g_fa2_noalloc_dq) != cudaSuccess || scratch == nullptr)
       return FA2_ERR_CUDA;
-    }
+    n.sched = static_cast<unsigned int*>(sched);
+    n.noalloc_dq = static_cast<float*>(scratch);
+    di = n;
   }
   *info = di;
   return FA2_OK;
@@ -221,27 +241,93 @@ fa2_status launched(int n) {
   return FA2_OK;
 }
 
-// Work counters of the packed forward's dynamic scheduler: pairs of
-// {next unit, finished CTAs}, zero between calls (each call's last CTA resets
-// its pair).  Calls take the pairs round robin, so up to kSchedSlots packed
-// forward calls may run at the same time on different streams.
-constexpr int kSchedSlots = 64;
-static __device__ unsigned int g_fa2_sched[2 * kSchedSlots];
-unsigned int* g_sched_addr[kMaxDevices] = {};
+// Work counters of the counter-scheduled calls (packed, block-sparse, and
+// padded backward calls with a causal mask over many key blocks): pairs
+// {next item, finished CTAs} in g_fa2_sched.  Each stream that makes such
+// calls owns one pair, so calls that may run at the same time (on different
+// streams) never share one, and calls on one stream, which run one after the
+// other, reuse it.  The pair is cleared on the call's stream right before
+// each launch (the call's last CTA clears it too), which also repairs a pair
+// that an aborted call left non-zero.  Up to kSchedSlots streams per device
+// own a pair at a time; a further stream takes over the pair used least
+// recently, after making itself wait (cudaStreamWaitEvent) for the event
+// recorded after that pair's last launch, so the two calls cannot overlap.
+// During stream capture nothing is recorded: the captured call keeps the
+// capturing stream's pair, and a hand-over that would need a wait is refused
+// (FA2_ERR_UNSUPPORTED).
+struct SchedSlots {
+  cudaStream_t owner[kSchedSlots] = {};
+  bool owned[kSchedSlots] = {};
+  uint64_t last_use[kSchedSlots] = {};
+  cudaEvent_t done[kSchedSlots] = {};  // recorded after the pair's last (uncaptured) launch
+  bool done_valid[kSchedSlots] = {};
+};
+SchedSlots g_slots[kMaxDevices];
 std::mutex g_sched_mu;
-std::atomic<uint32_t> g_sched_ticket{0};
+uint64_t g_sched_clock = 0;
 
-fa2_status sched_counters(int dev, unsigned int** out) {
-  {
-    std::lock_guard<std::mutex> lk(g_sched_mu);
-    if (g_sched_addr[dev] == nullptr) {
-      void* ptr = nullptr;
-      if (cudaGetSymbolAddress(&ptr, g_fa2_sched) != cudaSuccess || ptr == nullptr) return FA2_ERR_CUDA;
-      g_sched_addr[dev] = static_cast<unsigned int*>(ptr);
+// The counter pair of one launch.  acquire() takes the stream's pair and
+// clears it on the stream; finish(), called right after the launch, records
+// the pair's event.  The table stays locked in between, so the launch and
+// its event are ordered with every other stream's hand-over.
+class SchedLease {
+ public:
+  fa2_status acquire(int dev, const DeviceInfo& di, cudaStream_t st, unsigned int** out) {
+    lk_ = std::unique_lock<std::mutex>(g_sched_mu);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return FA2_ERR_CUDA;
+    capturing_ = cs != cudaStreamCaptureStatusNone;
+    SchedSlots& t = g_slots[dev];
+    int s = -1;
+    for (int i = 0; i < kSchedSlots && s < 0; ++i)
+      if (t.owned[i] && t.owner[i] == st) s = i;
+    for (int i = 0; i < kSchedSlots && s < 0; ++i)
+      if (!t.owned[i]) s = i;
+    if (s < 0) {  // every pair is owned: take over the least recently used one
+      s = 0;
+      for (int i = 1; i < kSchedSlots; ++i)
+        if (t.last_use[i] < t.last_use[s]) s = i;
+      if (t.done_valid[s]) {
+        if (capturing_) return FA2_ERR_UNSUPPORTED;
+        if (cudaStreamWaitEvent(st, t.done[s], 0) != cudaSuccess) return FA2_ERR_CUDA;
+      }
     }
+    if (!capturing_ && t.done[s] == nullptr &&
+        cudaEventCreateWithFlags(&t.done[s], cudaEventDisableTiming) != cudaSuccess)
+      return FA2_ERR_CUDA;
+    t.owner[s] = st;
+    t.owned[s] = true;
+    t.last_use[s] = ++g_sched_clock;
+    unsigned int* pair = di.sched + 2 * s;
+    if (cudaMemsetAsync(pair, 0, 2 * sizeof(unsigned int), st) != cudaSuccess) return FA2_ERR_CUDA;
+    dev_ = dev;
+    slot_ = s;
+    st_ = st;
+    *out = pair;
+    return FA2_OK;
   }
-  *out = g_sched_addr[dev] + 2 * (g_sched_ticket.fetch_add(1) % kSchedSlots);
-  return FA2_OK;
+  fa2_status finish() {
+    if (slot_ < 0) return FA2_OK;
+    SchedSlots& t = g_slots[dev_];
+    if (!capturing_) {
+      if (cudaEventRecord(t.done[slot_], st_) != cudaSuccess) return FA2_ERR_CUDA;
+      t.done_valid[slot_] = true;
+    }
+    slot_ = -1;
+    lk_.unlock();
+    return FA2_OK;
+  }
+
+ private:
+  std::unique_lock<std::mutex> lk_;
+  int dev_ = -1, slot_ = -1;
+  cudaStream_t st_ = nullptr;
+  bool capturing_ = false;
+};
+
+DeviceInfo device_info(int dev) {
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  return g_dev[dev];
 }
 
 template <int HD>
@@ -290,7 +376,9 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.bm_sb = a.bm_sb;
   p.bm_sh = a.bm_sh;
   p.nb = (a.N + 127) / 128;
-  if (MODE != kLayoutPadded) FA2_TRY(sched_counters(dev, &p.sched));
+  p.test_skip = g_test_skip.load() == 1;
+  SchedLease lease;
+  if (MODE != kLayoutPadded) FA2_TRY(lease.acquire(dev, device_info(dev), st, &p.sched));
   auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, MODE, FP8>;
   constexpr int smem = FwdCfg<HD, FP8>::SMEM_BYTES;
   FA2_TRY(ensure_smem(kern, smem, dev, mask));
@@ -305,7 +393,8 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   // persistent grid: one CTA per SM (shared memory and TMEM allow one)
   const unsigned grid = unsigned(std::min(p.num_units, std::max(sm_count, 1)));
   kern<<<grid, FwdCfg<HD, FP8>::THREADS, smem, st>>>(p);
-  return launched(1);
+  FA2_TRY(launched(1));
+  return lease.finish();
 }
 
 template <int HD, bool ALIBI, bool DROPOUT, int MODE>
@@ -314,7 +403,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
                             const fa2_strides& sdk, const fa2_strides& sdv, int deterministic,
                             int dev, cudaStream_t st) {
   static std::atomic<uint64_t> mask_dkdv{0}, mask_dkdv_nodq{0}, mask_dq{0};
-  static std::atomic<uint64_t> mask_dkdv_dyn{0}, mask_dkdv_nodq_dyn{0};
+  static std::atomic<uint64_t> mask_dkdv_dyn{0}, mask_dkdv_nodq_dyn{0}, mask_dkdv_ord{0};
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
   const MapShape ms = map_shape(a);
@@ -325,7 +414,13 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   FA2_TRY(encode_input(&p.tm_dq, a.dq, sdq, a, HD));
   FA2_TRY(encode_input(&p.tm_dk, a.dk, sdk, a, HD));
   FA2_TRY(encode_input(&p.tm_dv, a.dv, sdv, a, HD));
-  if (!deterministic) FA2_TRY(encode_dqacc_3d(&p.tm_dqacc, a.dq_accum, ms.bt, ms.rows, a.H, HD));
+  // Deterministic calls under a causal mask (padded layout) add dQ in a
+  // fixed order inside the dK/dV kernel; other deterministic calls run the
+  // ordered second pass (kernel 2).
+  constexpr bool CAN_DYN = MODE == kLayoutPadded;
+  const bool ordered = CAN_DYN && deterministic && a.wr == 0;
+  const bool accumulate = !deterministic || ordered;  // dQ through the fp32 accumulator
+  if (accumulate) FA2_TRY(encode_dqacc_3d(&p.tm_dqacc, a.dq_accum, ms.bt, ms.rows, a.H, HD));
   p.dq = static_cast<__nv_bfloat16*>(a.dq);
   p.dk = static_cast<__nv_bfloat16*>(a.dk);
   p.dv = static_cast<__nv_bfloat16*>(a.dv);
@@ -353,6 +448,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.wait_ns = g_wait_ns.load();
   p.drop = a.drop;
+  p.test_skip = g_test_skip.load() == 2;
   const unsigned grid = unsigned(p.nblocks) * unsigned(a.H) * unsigned(a.B);
   // kernel 1 is persistent: one CTA per SM walks the work items
   p.num_items = int(grid);
@@ -369,12 +465,17 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   // order.  Measured (d = 128, B N = 16384): the counter wins from 128 key
   // blocks on (N = 16384: +9 %; d = 64: +5 %; window (4096, 0) at N = 32768:
   // +1 %) and loses below (N = 4096: -3 %, N = 8192: -5 %).
-  constexpr bool CAN_DYN = MODE == kLayoutPadded;
-  const bool dyn = CAN_DYN && a.wr == 0 && p.nblocks >= 128;
-  if (MODE != kLayoutPadded || dyn) FA2_TRY(sched_counters(dev, &p.sched));
+  // The ordered dQ needs the counter schedule (its key blocks are taken in
+  // a fixed order as CTAs become free).
+  const bool dyn = CAN_DYN && a.wr == 0 && (p.nblocks >= 128 || ordered);
+  SchedLease lease;
+  if (MODE != kLayoutPadded || dyn) FA2_TRY(lease.acquire(dev, di, st, &p.sched));
+  const size_t accum_floats = size_t(ms.bt) * a.H * ms.rows * HD;
+  if (ordered) p.dq_chain = reinterpret_cast<uint32_t*>(a.dq_accum + accum_floats);
   using K1 = void (*)(BwdParams);
-  const K1 k1_dq = dyn ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE, CAN_DYN>
-                       : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE>;
+  const K1 k1_dq = ordered ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE, CAN_DYN, CAN_DYN>
+                   : dyn   ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE, CAN_DYN>
+                           : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE>;
   const K1 k1_nodq = dyn ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, MODE, CAN_DYN>
                          : fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, false, DROPOUT, MODE>;
   constexpr int smem1 = BwdCfg<HD>::SMEM_BYTES;
@@ -384,17 +485,19 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   // forever.  Refuse to launch otherwise.
   {
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, deterministic ? k1_nodq : k1_dq) != cudaSuccess) return FA2_ERR_CUDA;
+    if (cudaFuncGetAttributes(&fa, accumulate ? k1_dq : k1_nodq) != cudaSuccess) return FA2_ERR_CUDA;
     if (fa.numRegs < BwdCfg<HD>::REGS_AT_LAUNCH) return FA2_ERR_UNSUPPORTED;
   }
-  if (!deterministic) {
-    const long long n4 = (long long)ms.bt * a.H * ms.rows * HD / 4;
+  if (accumulate) {
+    // clear the accumulator (and the ordered dQ's counters, which follow it)
+    const long long n4 = (long long)(accum_floats + (ordered ? size_t(ms.bt) * a.H * p.nblocks * 4 : 0)) / 4;
     const unsigned zgrid = unsigned(std::min<long long>((n4 + 255) / 256, 148 * 16));
     zero_f32x4_kernel<<<zgrid, 256, 0, st>>>(reinterpret_cast<float4*>(a.dq_accum), n4);
     FA2_TRY(launched(1));
-    FA2_TRY(ensure_smem(k1_dq, smem1, dev, dyn ? mask_dkdv_dyn : mask_dkdv));
+    FA2_TRY(ensure_smem(k1_dq, smem1, dev, ordered ? mask_dkdv_ord : dyn ? mask_dkdv_dyn : mask_dkdv));
     k1_dq<<<grid1, BwdCfg<HD>::THREADS, smem1, st>>>(p);
     FA2_TRY(launched(1));
+    FA2_TRY(lease.finish());
     AttnArgs c = a;  // the accumulator is [bt * H, rows, d] in both layouts
     c.B = ms.bt;
     c.N = ms.rows;
@@ -407,6 +510,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   FA2_TRY(ensure_smem(k1_nodq, smem1, dev, dyn ? mask_dkdv_nodq_dyn : mask_dkdv_nodq));
   k1_nodq<<<grid1, BwdCfg<HD>::THREADS, smem1, st>>>(p);
   FA2_TRY(launched(1));
+  FA2_TRY(lease.finish());
   auto k2 = fa2_bwd_dq_sm100_kernel<HD, ALIBI, DROPOUT, MODE>;
   constexpr int smem2 = DqCfg<HD>::SMEM_BYTES;
   FA2_TRY(ensure_smem(k2, smem2, dev, mask_dq));
@@ -607,6 +711,12 @@ fa2_status fa2_set_wait_limit_ms(int ms) {
   return FA2_OK;
 }
 
+fa2_status fa2_test_skip_arrive(int which) {
+  if (which < 0 || which > 2) return FA2_ERR_INVALID_ARG;
+  g_test_skip.store(which);
+  return FA2_OK;
+}
+
 fa2_status fa2_device_status(int* code, int clear) {
   if (code == nullptr) return FA2_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return FA2_ERR_CUDA;
@@ -754,8 +864,11 @@ fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D, int B, 
 
 size_t fa2_bwd_workspace_size(int B, int N, int H, int d, fa2_dtype dtype, int deterministic) {
   if (check_shape(B, N, H, d, dtype) != FA2_OK) return 0;
-  if (dtype != FA2_BF16 || deterministic) return 0;
-  const size_t bytes = size_t(B) * H * N * d * sizeof(float);
+  if (dtype != FA2_BF16) return 0;
+  // fp32 dQ accumulator [B*H, N, d]; deterministic calls add one counter
+  // per 32-row box of every query block [B*H, ceil(N/128), 4]
+  size_t bytes = size_t(B) * H * N * d * sizeof(float);
+  if (deterministic) bytes += size_t(B) * H * ((N + 127) / 128) * 4 * sizeof(uint32_t);
   return (bytes + 255) & ~size_t(255);
 }
 
@@ -843,32 +956,9 @@ fa2_status fa2_bwd_blocksparse(const void* q, const void* k, const void* v, cons
 
 // ---------------------------------------------------------------------------
 // fa2_bwd_noalloc: fa2_bwd (bf16, non-deterministic) with its fp32 dQ
-// accumulator in a fixed device array instead of caller workspace.
+// accumulator in a fixed device array (g_fa2_noalloc_dq above) instead of
+// caller workspace.
 // ---------------------------------------------------------------------------
-}  // extern "C"
-
-namespace {
-// The scratch array.  In host code this name is only a stand-in for the
-// device object: its device address comes from cudaGetSymbolAddress, looked
-// up once per device with that device current.
-static __device__ __align__(256) float g_fa2_noalloc_dq[FA2_NOALLOC_MAX_DQ_FLOATS];
-float* g_noalloc_addr[kMaxDevices] = {};
-std::mutex g_noalloc_mu;
-
-fa2_status noalloc_scratch(int dev, float** out) {
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_fa2_noalloc_dq) != cudaSuccess || ptr == nullptr)
-      return FA2_ERR_CUDA;
-    g_noalloc_addr[dev] = static_cast<float*>(ptr);
-  }
-  *out = g_noalloc_addr[dev];
-  return FA2_OK;
-}
-}  // namespace
-
-extern "C" {
 
 fa2_status fa2_bwd_noalloc(const void* q, const void* k, const void* v, const void* dout,
                            const float* lse, const float* D, void* dq, void* dk, void* dv, int B,
@@ -894,8 +984,7 @@ fa2_status fa2_bwd_noalloc(const void* q, const void* k, const void* v, const vo
   DeviceInfo di;
   FA2_TRY(current_device(&dev, &di));
   if (di.sm_major != 10 || di.sm_minor != 0) return FA2_ERR_UNSUPPORTED;
-  float* scratch = nullptr;
-  FA2_TRY(noalloc_scratch(dev, &scratch));
+  float* scratch = di.noalloc_dq;  // device address of the fixed scratch array
   AttnArgs a;  // the scratch is cleared by the first kernel of the launch sequence
   fill_bwd_args(&a, q, k, v, dout, lse, D, dq, dk, dv, scratch, B, N, H, d, sq, sk, sv, sdo, sdq,
                 sdk, sdv, softmax_scale, causal, window_left, window_right, alibi_slopes, 0.f, 0);

@@ -101,6 +101,37 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, AbortFla
   return wait_bar_slow(bar, parity, ab, limit_ns, site);
 }
 
+// Global-memory counters shared between CTAs (acquire / release at GPU
+// scope), and a bounded wait for a counter to reach a value: like wait_bar,
+// it gives up (recording `site`) after `limit_ns` or when the CTA's abort
+// flag is set.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool wait_counter_eq(const uint32_t* p, uint32_t value, AbortFlag ab,
+                                                uint64_t limit_ns, int site) {
+  if (ld_acquire_gpu(p) == value) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(p) == value) return true;
+    if ((it & 15u) == 0) {
+      if (*ab.flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *ab.flag = 1;
+        atomicCAS(&g_fa2_device_status, 0, site);
+        __threadfence();
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast anywhere.
 // ---------------------------------------------------------------------------
@@ -157,6 +188,12 @@ __device__ __forceinline__ void bulk_wait_all() {
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order global-memory accesses of the generic proxy (counters) and of the
+// async proxy (TMA reductions) made by this thread.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Named barrier over `count` threads (a multiple of 32).

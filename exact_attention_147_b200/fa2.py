@@ -40,7 +40,8 @@ EXPORTED = ("fa2_fwd", "fa2_bwd_preprocess", "fa2_bwd_workspace_size", "fa2_bwd"
             "fa2_fwd_varlen", "fa2_bwd_varlen", "fa2_fwd_blocksparse", "fa2_bwd_blocksparse",
             "fa2_fwd_fp8",
             "fa2_strerror", "fa2_device_status",
-            "fa2_set_wait_limit_ms", "fa2_kernel_launches", "fa2_bwd_noalloc")
+            "fa2_set_wait_limit_ms", "fa2_kernel_launches", "fa2_bwd_noalloc",
+            "fa2_test_skip_arrive")
 # Device status code of a packed call whose cu_seqlens was malformed.
 STATUS_BAD_SEQLENS = 0xF10
 
@@ -103,6 +104,8 @@ def load_library(path: str = LIB_PATH):
     lib.fa2_device_status.restype = i
     lib.fa2_set_wait_limit_ms.argtypes = [i]
     lib.fa2_set_wait_limit_ms.restype = i
+    lib.fa2_test_skip_arrive.argtypes = [i]
+    lib.fa2_test_skip_arrive.restype = i
     lib.fa2_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
                                     s, s, s, s, s, s, s, f, i, i, i, vp, f, vp]
     lib.fa2_bwd_noalloc.restype = i
@@ -396,6 +399,12 @@ def kernel_launches() -> int:
 
 def set_wait_limit_ms(ms: int):
     _check(load_library().fa2_set_wait_limit_ms(int(ms)), "fa2_set_wait_limit_ms")
+
+
+def test_skip_arrive(which: int):
+    """Test switch of the bounded-wait path: 1 = forward, 2 = backward, 0 = off
+    (see fa2_test_skip_arrive in include/fa2.h)."""
+    _check(load_library().fa2_test_skip_arrive(int(which)), "fa2_test_skip_arrive")
 
 
 class _Fa2Function(torch.autograd.Function):

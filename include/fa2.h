@@ -35,12 +35,25 @@
  *  - All pointers are DEVICE pointers, owned by the caller; the library
  *    allocates no device memory and keeps no state between calls except a
  *    small cache of device properties, the device status word read by
- *    fa2_device_status(), and a table of 64 work counters.  Calls whose work
- *    items differ in cost (the *_varlen and *_blocksparse calls, and
- *    backward calls with a causal mask over 128 or more key blocks) take
- *    their items from one of these counters, in turn, and the last CTA of
- *    the call resets it.  At most 64 such calls may therefore run at the
- *    same time on one device (on different streams).
+ *    fa2_device_status(), a table of 64 work-counter pairs per device and
+ *    the scratch array of fa2_bwd_noalloc.  The first call that reaches a
+ *    device looks up the device addresses of the last two
+ *    (cudaGetSymbolAddress, with that device current); make that first
+ *    call before any stream capture.
+ *  - Work counters.  Calls whose work items differ in cost (the *_varlen
+ *    and *_blocksparse calls, and backward calls with a causal mask over
+ *    128 or more key blocks) take their items from a counter pair.  Each
+ *    stream that makes such calls owns one pair: calls on one stream run in
+ *    order and reuse it, calls on different streams never share one while
+ *    both may run.  The pair is cleared on the call's stream before each
+ *    launch.  Up to 64 streams per device own a pair at a time; a further
+ *    stream takes over the least recently used pair after waiting, on the
+ *    GPU (an event), for that pair's last call to finish.  During stream
+ *    capture no such wait can be recorded: a captured call keeps the pair
+ *    of the capturing stream (a hand-over that would need a wait returns
+ *    FA2_ERR_UNSUPPORTED), and the caller must not replay the graph while
+ *    another call on the same pair runs (for instance the same graph on
+ *    two streams at once).
  *  - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
  *    default stream); nothing is synchronised.
  *  - Every argument is checked before anything is launched.  An invalid
@@ -134,23 +147,49 @@ fa2_status fa2_fwd(const void* q, const void* k, const void* v, void* o, float* 
  * Backward pre-processing: D[b, h, i] = sum_c dO[b, i, h, c] * O[b, i, h, c]
  * in fp32 (the row sums of dO o O that the softmax gradient needs).
  *
+ * The backward pass keeps only per-row statistics of the forward and
+ * rebuilds the scores on chip (explainer "AI基础 | Flash Attention",
+ * "Backward pass"); with P the softmax, the gradient of the scores is
+ * dS_ij = P_ij (dP_ij - D_i), dP = dO V^T, where D_i = sum_j P_ij dP_ij
+ * equals sum_c dO_ic O_ic because O = P V.  This call computes D from O
+ * and dO, so the backward kernels never form a row of dP in full before
+ * they can use it.
+ *
  *   o, dout  [B, N, H, d] (dtype), strides so, sdo.
  *   D        [B, H, N] fp32 output, dense.
+ *
+ * Unlike a common layout of this step, the call does not clear the fp32 dQ
+ * accumulator: fa2_bwd clears its own workspace before it adds into it, so
+ * the workspace's contents on entry never matter.
  */
 fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D,
                               int B, int N, int H, int d, fa2_dtype dtype,
                               fa2_strides so, fa2_strides sdo, void* stream);
 
 /*
- * Bytes of device workspace fa2_bwd needs for these shapes (an fp32 dQ
- * accumulator for bf16, nothing for fp32).  The caller allocates it; its
- * contents on entry do not matter.  Returns 0 for invalid shapes.
+ * Bytes of device workspace fa2_bwd needs for these shapes: for bf16, an fp32
+ * dQ accumulator (B * H * N * d floats) and, when deterministic, one 32-bit
+ * counter per 32 query rows (B * H * ceil(N / 128) * 4); nothing for fp32.
+ * The caller allocates it; its contents on entry do not matter (the call
+ * clears what it uses).  Returns 0 for invalid shapes.
  */
 size_t fa2_bwd_workspace_size(int B, int N, int H, int d, fa2_dtype dtype, int deterministic);
 
 /*
  * Backward pass: dQ, dK, dV of L = sum(O o dO) given the forward's lse and
- * the pre-processed D.  The probabilities are recomputed from q, k and lse.
+ * the pre-processed D.  The probabilities are recomputed from q, k and lse
+ * (explainer "AI基础 | Flash Attention", "Backward pass": the N x N matrices
+ * are not stored; only the per-row statistics are, and the scores are
+ * rebuilt block by block on chip).  The pages print no gradient formulas;
+ * the ones computed are the textbook softmax and matrix-product gradients,
+ * with c = softmax_scale:
+ *     P = exp(c Q K^T + bias - LSE),  dV = P^T dO,  dP = dO V^T,
+ *     dS = P o (dP - D),  dQ = c dS K,  dK = c dS^T Q.
+ * Work is split over key blocks of every (batch, head) (FlashAttention-2
+ * abstract, arXiv 2307.08691: parallelism across thread blocks within a
+ * head); dQ partial sums of different key blocks are added in fp32.  The
+ * `deterministic` option is the one of the call in the "FlashAttention v2"
+ * article, §5.1-§5.2.
  *
  *   q, k, v, dout    [B, N, H, d] inputs (dtype) with strides sq, sk, sv, sdo.
  *   lse, D           [B, H, N] fp32 from fa2_fwd and fa2_bwd_preprocess.
@@ -161,9 +200,13 @@ size_t fa2_bwd_workspace_size(int B, int N, int H, int d, fa2_dtype dtype, int d
  *   dropout_p, dropout_seed
  *                    exactly as passed to fa2_fwd.
  *   deterministic    0: dQ partial sums from different key blocks are added
- *                    with fp32 atomics (fast, order not fixed);
- *                    nonzero: dQ is produced by an ordered pass with no
- *                    atomics, so dq, dk and dv are bitwise repeatable.
+ *                    with fp32 reductions in whatever order they arrive
+ *                    (fast, bits may differ between runs);
+ *                    nonzero: dq, dk and dv are bitwise repeatable.  Under a
+ *                    causal mask (window_right = 0) the partial sums of each
+ *                    query block are added in a fixed order (descending key
+ *                    block) inside the same kernel; otherwise dQ comes from
+ *                    a second, ordered pass that recomputes the scores.
  */
 fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout,
                    const float* lse, const float* D, void* dq, void* dk, void* dv,
@@ -318,9 +361,10 @@ fa2_status fa2_fwd_fp8(const void* q, const void* k, const void* v, void* o, flo
  *   Limit:   B * H * N * d must not exceed FA2_NOALLOC_MAX_DQ_FLOATS;
  *            larger problems return FA2_ERR_SCRATCH_LIMIT and launch
  *            nothing (use fa2_bwd with a workspace instead).
- *   Set-up:  the first call on a device looks up the device address of the
- *            array (cudaGetSymbolAddress) with that device current; make
- *            that first call before any stream capture.
+ *   Set-up:  the device address of the array is looked up
+ *            (cudaGetSymbolAddress, with the device current) by the first
+ *            call of any entry point that reaches the device; make that
+ *            first call before any stream capture.
  *   Sharing: every call on a device uses the same array.  The accumulator
  *            is cleared at the start of each call, but two calls whose
  *            kernels overlap on the GPU (different streams, no ordering
@@ -355,6 +399,23 @@ fa2_status fa2_device_status(int* code, int clear);
  * < 1 are rejected with FA2_ERR_INVALID_ARG.
  */
 fa2_status fa2_set_wait_limit_ms(int ms);
+
+/*
+ * Test switch for the bounded-wait path (0 in normal use, the default).
+ * With which = 1 every later forward launch of the tensor-core kernels, and
+ * with which = 2 every later backward launch (the dK/dV kernel), has the
+ * CTA that takes work item 0 (a query-tile pair, or a key block, of batch 0
+ * and head 0; the first item that CTA takes) withhold one mbarrier arrive
+ * on its first block, so that the MMA warp's wait for it runs out after the
+ * limit set by fa2_set_wait_limit_ms.  That CTA then records the wait's
+ * site code in the device status word, its other roles give up their own
+ * waits through the CTA's abort flag, it waits (again with a limit) for the
+ * copies and products it has in flight, frees its tensor memory and exits;
+ * the other CTAs finish normally.  The outputs of such a call are unspecified;
+ * fa2_device_status reports FA2_ERR_DEVICE_TIMEOUT.  Set 0 to switch it
+ * off.  Returns FA2_ERR_INVALID_ARG for other values.
+ */
+fa2_status fa2_test_skip_arrive(int which);
 
 /*
  * Number of kernels this library has launched in this process since it was

@@ -28,3 +28,18 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _device_status_word(request):
+    """GPU tests start with a clear device status word and must leave it
+    clear: a kernel that gave up a bounded wait is reported against the test
+    that launched it, not a later one."""
+    if "gpu" not in request.keywords:
+        yield
+        return
+    from exact_attention_147_b200 import fa2 as F
+    F.device_status(clear=True)
+    yield
+    code = F.device_status(clear=True)
+    assert code == 0, f"device status {code:#x} left by this test"

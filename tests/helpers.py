@@ -142,3 +142,17 @@ def fp8_o_bound(q, k, v, scale, causal=False, wl=-1, wr=-1, slope=None):
     err_p = np.where(P > 0, np.maximum(2.0 ** -4 * P, 2.0 ** -10), 0.0)
     o = (P @ v) / l
     return (err_p @ np.abs(v)) / l + 2.0 ** -8 * np.abs(o) + 1e-6 * (P @ np.abs(v)) / l
+
+
+def assert_same_sum_any_order(a: torch.Tensor, b: torch.Tensor, what: str = ""):
+    """a and b are bf16 roundings of fp32 sums of the same partial terms added
+    in two different fixed orders (e.g. the deterministic dQ of the ordered
+    in-kernel chain and of the second pass).  The fp32 sums differ only by
+    reordering, far below one bf16 step, so the rounded values differ by at
+    most one bf16 step (2^-7 relative) -- plus, where the sum cancels to near
+    zero, a small absolute term (2^-12 of the largest value)."""
+    a64, b64 = a.double(), b.double()
+    bound = 2.0 ** -7 * b64.abs() + 2.0 ** -12 * float(b64.abs().max())
+    diff = (a64 - b64).abs()
+    assert bool((diff <= bound).all()), (
+        f"{what}: max diff {float(diff.max()):.3e} beyond one bf16 step")

@@ -63,3 +63,18 @@ def test_captured_traffic_follows_the_source_hash(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(fake_root))
     assert bench.captured_traffic("fa2_fwd") == 123
     assert bench.captured_traffic("fa2_bwd") is None
+
+
+def test_reference_arm_prints_the_gpu_arms_config(monkeypatch, capsys):
+    # the two arms must describe the same workload with the same dict, and
+    # the reference's ms_per_step is the time it measured, not an estimate
+    import argparse
+    monkeypatch.setattr(bench, "REF_STEP_S", 0.0)
+    monkeypatch.delenv("RANK", raising=False)
+    assert bench.run_reference(argparse.Namespace(steps=1, warmup=0)) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["config"] == bench.bench_config(bench.WORKLOAD)
+    assert line["impl"] == "reference"
+    assert 0 < line["ms_per_step"] < line["ms_per_full_step_extrapolated"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0

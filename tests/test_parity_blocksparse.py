@@ -141,7 +141,13 @@ def test_all_ones_mask_equals_padded_kernels_bitwise(causal):
     g = F.bwd(do, q, k, v, l2, D, causal=causal, deterministic=True)
     torch.cuda.synchronize()
     assert torch.equal(out, o2) and torch.equal(lse, l2)
-    assert torch.equal(dq, g[0]) and torch.equal(dk, g[1]) and torch.equal(dv, g[2])
+    assert torch.equal(dk, g[1]) and torch.equal(dv, g[2])
+    if causal:
+        # the padded causal call adds dQ in its in-kernel order (descending key
+        # block), the block-sparse one in its second pass (ascending)
+        assert_same_sum_any_order(dq, g[0], "dq")
+    else:
+        assert torch.equal(dq, g[0])
 
 
 def test_local_global_pattern_bench_size():

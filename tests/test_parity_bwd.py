@@ -4,6 +4,8 @@ The GPU runs its own forward (for LSE and O), bwd_preprocess and bwd; the
 oracle recomputes every gradient from the same inputs.
 """
 
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -82,18 +84,33 @@ def test_mid_sampled(causal):
     compare_heads(w, [(0, 0), (w.B - 1, w.H - 1)])
 
 
-@pytest.mark.parametrize("n", [512, 4096, 16384])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n", W.SWEEP_N)
 @pytest.mark.parametrize("d", [128, 64])
-def test_sweep_sampled(n, d):
-    w = W.sweep(n, d, causal=(n == 4096))
+def test_sweep_sampled(n, d, causal):
+    # every point of the sequence-length sweep (hidden 2048 as H=16 x d=128
+    # and as H=32 x d=64), one whole head each
+    w = W.sweep(n, d, causal)
     compare_heads(w, [(w.B - 1, w.H - 1)])
 
 
-def test_causal_long_sampled():
+@pytest.mark.parametrize("d", [128, 64])
+def test_causal_long_sampled(d):
     # 128 key blocks under a causal mask: the dK/dV kernel takes its items
-    # from the shared counter
-    w = W.sweep(16384, 128, causal=True)
-    compare_heads(w, [(0, w.H - 1)])
+    # from the shared counter (both head dims), first and last heads
+    w = W.sweep(16384, d, causal=True)
+    compare_heads(w, [(0, 0), (0, w.H - 1)])
+
+
+@pytest.mark.parametrize("n,causal", [(1024, False), (4096, True), (16384, True)])
+def test_deterministic_d64(n, causal):
+    # the padded-layout ordered dQ pass at d = 64: parity on a sampled head
+    # and bitwise-identical dq, dk, dv across two runs
+    w = dataclasses.replace(W.sweep(n, 64, causal), deterministic=True)
+    dq1, dk1, dv1 = compare_heads(w, [(w.B - 1, w.H - 1)])
+    q, k, v, do = W.make_inputs(w, "cuda")
+    _, _, dq2, dk2, dv2 = run_fwd_bwd(w, q, k, v, do)
+    assert torch.equal(dq1, dq2) and torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
 
 
 def test_long_local_sampled():
