@@ -69,7 +69,7 @@ struct BwdParams {
   DropoutParams drop;                    // used by the DROPOUT instantiations
   int num_items;                         // key blocks x heads x batch (kernel 1 work items)
   unsigned int* sched;                   // packed / block-sparse kernel 1: {next item, finished CTAs}
-  uint32_t* dq_chain;                    // ordered dQ: [B*H, nblocks, 4] counters (zero at launch)
+  uint32_t* dq_chain;                    // ordered dQ: [2, B*H, nblocks, 4] counters (zero at launch)
   int test_skip;                         // test switch, 0 in normal use: see kernel 1's ds_ready arrive
 };
 
@@ -298,6 +298,15 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   constexpr bool DYN = PACKED || SPARSE || DSCHED;  // items taken from the shared counter
   using namespace bwd_detail;
   constexpr int QS = C::Q_STAGES, DS = C::DO_STAGES;
+  // Register split.  The ordered dQ's drain holds a whole 128-column fp32
+  // tile and the chain state, so (without a dropout mask in the compute
+  // warps, which need their registers then) it takes 16 registers from the
+  // compute warpgroups: 128 / 152 / 104, no spills.
+  constexpr bool DRAIN_HEAVY = ORDER && !DROPOUT;
+  constexpr int REGS_CMP = DRAIN_HEAVY ? C::REGS_COMPUTE - 8 : C::REGS_COMPUTE;
+  constexpr int REGS_DRN = DRAIN_HEAVY ? C::REGS_DRAIN + 16 : C::REGS_DRAIN;
+  static_assert(2 * 128 * REGS_CMP + 128 * REGS_DRN + 128 * C::REGS_MISC == 512 * C::REGS_AT_LAUNCH,
+                "register split must use exactly the launch budget");
   constexpr int NCH = HD / 64;
   constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + HD;
 
@@ -610,7 +619,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       }
     }
   } else if (wg < 2) {
-    regs_inc<C::REGS_COMPUTE>();
+    regs_inc<REGS_CMP>();
     // ------------------------------------------------------------ compute (key rows)
     const int r = (warp % 4) * 32 + lane;
     const int cq = 64 * wg;  // this warpgroup's query columns [cq, cq + 64)
@@ -808,7 +817,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       ++jn;
     }
   } else {
-    regs_inc<C::REGS_DRAIN>();
+    regs_inc<REGS_DRN>();
     if (WITH_DQ) {
       // ---------------------------------------------------------- dQ drain (query rows)
       const int q = (warp % 4) * 32 + lane;
@@ -816,20 +825,8 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       const int wq = warp % 4;
       int g = 0, k = 0;
       bool ok = true;
-      // Ordered dQ: the box (this warp's 32 rows of a query block) whose adds
-      // were issued last and whose counter is still to be raised.
-      long long pend_box = -1;
+      long long pend_box = -1;  // ordered dQ: the box whose adds are in flight
       uint32_t pend_val = 0;
-      auto chain_release = [&]() {
-        if (ORDER && pend_box >= 0) {
-          if (lane == 0) {
-            bulk_wait_all();              // this warp's adds into the box are complete
-            fence_proxy_async_global();
-            st_release_gpu(p.dq_chain + pend_box, pend_val);
-          }
-          pend_box = -1;
-        }
-      };
       for (;;) {
         int I;
         ok = next_item(k, I, true, SITE_BRED + 1);
@@ -851,7 +848,8 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           // the slots free up.  Each warp stages its own 32 rows (a 32 x
           // 32-column box, 4 KB) and issues the bulk reduction for them: no
           // cross-warp barrier.
-          auto stage = [&](const uint32_t (&u)[32], int chunk) {
+          // acc: which of the ordered dQ's two accumulators (0 otherwise)
+          auto stage = [&](const uint32_t (&u)[32], int chunk, int acc) {
             if (lane == 0) bulk_wait_read_1();   // this warp's previous box in the slot was read
             __syncwarp();
             uint8_t* row = sStg + (chunk & 1) * 16384 + q * 128;
@@ -863,7 +861,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
             __syncwarp();
             if (lane == 0) {
               tma_reduce_add_3d(&p.tm_dqacc, smem_u32(sStg + (chunk & 1) * 16384 + wq * 4096), chunk * 32,
-                                itm.trow + i0 + wq * 32, bh);
+                                itm.trow + i0 + wq * 32, bh + acc * p.B * p.H);
               bulk_commit();
             }
           };
@@ -875,19 +873,22 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
           tc_fence_before();
           bar_arrive(dq_free);   // TMEM columns may now take the next dP^T
           if (ORDER) {
-            // Deterministic dQ under a causal mask: every box takes the key
-            // blocks' partial sums in descending key-block order.  Key block
-            // kb reaches query block qb after qb - kb steps of its own walk,
-            // which is its rank in that order, and the key blocks of a head
-            // are taken last first, so a partial sum arrives about when its
-            // turn comes and only ever waits for items taken earlier (no
-            // wait can close a cycle).  The box's counter holds how many sums
-            // it has received: wait for our rank, add, and raise the counter
-            // once the adds are complete (at the next box, or at the end of
-            // the item).
-            chain_release();
-            const long long box = ((long long)bh * p.nblocks + qb) * 4 + wq;
-            const uint32_t rank = uint32_t(qb - itm.kb);
+            // Deterministic dQ under a causal mask.  The partial sums of a
+            // 32-row box go to one of two accumulators by the parity of the
+            // key block, and each accumulator takes them in descending
+            // key-block order: key block kb reaches query block qb after
+            // qb - kb steps of its own walk, two steps after kb + 2, the one
+            // before it in its chain, and the key blocks of a head are taken
+            // last first, so a box only ever waits for items taken earlier
+            // (no wait can close a cycle).  A counter per box and accumulator
+            // holds how many sums it has received: wait for our rank, add, and
+            // raise it once the adds are complete, which is checked after the
+            // next box's adds have been issued (or at the end of the item),
+            // so the drain keeps one box's adds in flight.
+            const int acc = itm.kb & 1;
+            const long long box =
+                ((long long)(acc * p.B * p.H + bh) * p.nblocks + qb) * 4 + wq;
+            const uint32_t rank = uint32_t(qb - itm.kb) >> 1;
             bool turn = true;
             if (lane == 0) {
               turn = wait_counter_eq(p.dq_chain + box, rank, ab, p.wait_ns, SITE_BRED + 3);
@@ -895,15 +896,30 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
             }
             ok = __shfl_sync(0xffffffffu, turn ? 1 : 0, 0) != 0;
             if (!ok) break;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) stage(u[c], c, acc);
+            if (lane == 0 && pend_box >= 0) {
+              bulk_wait_upto<NC>();  // the previous box's adds are complete
+              fence_proxy_async_global();
+              st_release_gpu(p.dq_chain + pend_box, pend_val);
+            }
             pend_box = box;
             pend_val = rank + 1u;
+            continue;
           }
 #pragma unroll
-          for (int c = 0; c < NC; ++c) stage(u[c], c);
+          for (int c = 0; c < NC; ++c) stage(u[c], c, 0);
         }
         if (!ok) break;
         g += itm.nq;
-        chain_release();
+        if (ORDER && pend_box >= 0) {  // the item's last box: release it now
+          if (lane == 0) {
+            bulk_wait_all();
+            fence_proxy_async_global();
+            st_release_gpu(p.dq_chain + pend_box, pend_val);
+          }
+          pend_box = -1;
+        }
       }
       if (lane == 0) bulk_wait_all();
     } else if (DYN) {

@@ -420,7 +420,9 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   constexpr bool CAN_DYN = MODE == kLayoutPadded;
   const bool ordered = CAN_DYN && deterministic && a.wr == 0;
   const bool accumulate = !deterministic || ordered;  // dQ through the fp32 accumulator
-  if (accumulate) FA2_TRY(encode_dqacc_3d(&p.tm_dqacc, a.dq_accum, ms.bt, ms.rows, a.H, HD));
+  // (the ordered dQ keeps two accumulators, stacked: [2 * B * H, N, d])
+  if (accumulate)
+    FA2_TRY(encode_dqacc_3d(&p.tm_dqacc, a.dq_accum, ordered ? 2 * ms.bt : ms.bt, ms.rows, a.H, HD));
   p.dq = static_cast<__nv_bfloat16*>(a.dq);
   p.dk = static_cast<__nv_bfloat16*>(a.dk);
   p.dv = static_cast<__nv_bfloat16*>(a.dv);
@@ -470,7 +472,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   const bool dyn = CAN_DYN && a.wr == 0 && (p.nblocks >= 128 || ordered);
   SchedLease lease;
   if (MODE != kLayoutPadded || dyn) FA2_TRY(lease.acquire(dev, di, st, &p.sched));
-  const size_t accum_floats = size_t(ms.bt) * a.H * ms.rows * HD;
+  const size_t accum_floats = size_t(ordered ? 2 : 1) * ms.bt * a.H * ms.rows * HD;
   if (ordered) p.dq_chain = reinterpret_cast<uint32_t*>(a.dq_accum + accum_floats);
   using K1 = void (*)(BwdParams);
   const K1 k1_dq = ordered ? fa2_bwd_dkdv_sm100_kernel<HD, ALIBI, true, DROPOUT, MODE, CAN_DYN, CAN_DYN>
@@ -490,7 +492,7 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   }
   if (accumulate) {
     // clear the accumulator (and the ordered dQ's counters, which follow it)
-    const long long n4 = (long long)(accum_floats + (ordered ? size_t(ms.bt) * a.H * p.nblocks * 4 : 0)) / 4;
+    const long long n4 = (long long)(accum_floats + (ordered ? size_t(2) * ms.bt * a.H * p.nblocks * 4 : 0)) / 4;
     const unsigned zgrid = unsigned(std::min<long long>((n4 + 255) / 256, 148 * 16));
     zero_f32x4_kernel<<<zgrid, 256, 0, st>>>(reinterpret_cast<float4*>(a.dq_accum), n4);
     FA2_TRY(launched(1));
@@ -504,7 +506,9 @@ fa2_status launch_bwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
     c.cu_seqlens = nullptr;
     const long long rows = (long long)c.B * c.H * c.N;
     const long long per_block = 256 / (HD / 4);
-    dq_convert_kernel<HD><<<unsigned((rows + per_block - 1) / per_block), 256, 0, st>>>(c);
+    const unsigned cgrid = unsigned((rows + per_block - 1) / per_block);
+    if (ordered) dq_convert_kernel<HD, 2><<<cgrid, 256, 0, st>>>(c);
+    else dq_convert_kernel<HD><<<cgrid, 256, 0, st>>>(c);
     return launched(1);
   }
   FA2_TRY(ensure_smem(k1_nodq, smem1, dev, dyn ? mask_dkdv_nodq_dyn : mask_dkdv_nodq));
@@ -865,10 +869,11 @@ fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D, int B, 
 size_t fa2_bwd_workspace_size(int B, int N, int H, int d, fa2_dtype dtype, int deterministic) {
   if (check_shape(B, N, H, d, dtype) != FA2_OK) return 0;
   if (dtype != FA2_BF16) return 0;
-  // fp32 dQ accumulator [B*H, N, d]; deterministic calls add one counter
-  // per 32-row box of every query block [B*H, ceil(N/128), 4]
-  size_t bytes = size_t(B) * H * N * d * sizeof(float);
-  if (deterministic) bytes += size_t(B) * H * ((N + 127) / 128) * 4 * sizeof(uint32_t);
+  // fp32 dQ accumulator [B*H, N, d]; deterministic calls keep two of them
+  // and a counter per 32-row box of every query block for each,
+  // [2, B*H, ceil(N/128), 4]
+  size_t bytes = size_t(deterministic ? 2 : 1) * B * H * N * d * sizeof(float);
+  if (deterministic) bytes += size_t(2) * B * H * ((N + 127) / 128) * 4 * sizeof(uint32_t);
   return (bytes + 255) & ~size_t(255);
 }
 

@@ -123,9 +123,11 @@ struct FwdCfg {
   static constexpr int THREADS = 512;
   // registers per thread after re-balancing (launch: 128 x 512 = 65536):
   // softmax warpgroups 184, epilogue warpgroup 80, loader / MMA warpgroup 64
-  // (d = 64: 200 / 56 / 56, the split at which none of the roles spills)
-  static constexpr int REGS_SOFT = HD == 128 ? 184 : 200, REGS_EPI = HD == 128 ? 80 : 56,
-                       REGS_MISC = HD == 128 ? 64 : 56;
+  // (d = 64: 200 / 48 / 64 -- none of the roles spills, and the MMA issuer,
+  // whose latency from a finished P to the next S product the softmax
+  // waits on, measured about 1% faster with 64 than with 56)
+  static constexpr int REGS_SOFT = HD == 128 ? 184 : 200, REGS_EPI = HD == 128 ? 80 : 48,
+                       REGS_MISC = 64;
   static constexpr int REGS_AT_LAUNCH = (2 * 128 * REGS_SOFT + 128 * REGS_EPI + 128 * REGS_MISC) / 512;
   static_assert(REGS_AT_LAUNCH == 128, "register split must use exactly the launch budget");
 };
@@ -167,30 +169,7 @@ __device__ __forceinline__ bool pair_needs(const uint8_t* r0, const uint8_t* r1,
 // LSE = -inf from one fully hidden block).
 struct Unit {
   int h, b, bt, base, len, row0, first, last, nblk;
-  // blocks of the unit (relative to `first`) that each query tile needs:
-  // tile 0 [0, z0], tile 1 [a1, nblk - 1].  Under a causal or right-window
-  // mask tile 0 skips the unit's last block(s), under a left window tile 1
-  // skips its first, where every score of that tile would be hidden.
-  int z0, a1;
 };
-// Is relative block `it` of unit u one that query tile t needs?  (With a
-// block mask both tiles visit every block of the unit.)
-template <int MODE>
-__device__ __forceinline__ bool tile_needs(const Unit& u, int t, int it) {
-  if (MODE == kLayoutSparse) return true;
-  return t == 0 ? it <= u.z0 : it >= u.a1;
-}
-// Number of blocks of unit u that query tile t visits, and the first one.
-template <int MODE>
-__device__ __forceinline__ int tile_blocks(const Unit& u, int t) {
-  if (MODE == kLayoutSparse) return u.nblk;
-  return t == 0 ? u.z0 + 1 : u.nblk - u.a1;
-}
-template <int MODE>
-__device__ __forceinline__ int tile_first(const Unit& u, int t) {
-  if (MODE == kLayoutSparse) return 0;
-  return t == 0 ? 0 : u.a1;
-}
 template <int MODE>
 __device__ __forceinline__ Unit unit_of(const FwdParams& p, int L) {
   constexpr bool PACKED = MODE == kLayoutPacked;
@@ -220,8 +199,6 @@ __device__ __forceinline__ Unit unit_of(const FwdParams& p, int L) {
   u.first = 0;
   u.last = -1;
   u.nblk = 0;
-  u.z0 = -1;
-  u.a1 = 0;
   if (u.row0 < u.len) {
     const int row_end = min(u.len, u.row0 + 256);
     const int kv_lo = p.wl >= 0 ? max(0, u.row0 - p.wl) : 0;
@@ -244,18 +221,6 @@ __device__ __forceinline__ Unit unit_of(const FwdParams& p, int L) {
       } else {
         u.nblk = 1;
       }
-    }
-    // Blocks of each tile: both tiles visit every block of the unit, except
-    // that with both tiles holding rows of the sequence (and no block mask,
-    // which hides blocks element-wise instead) each visits only the blocks
-    // its own rows can see.
-    u.z0 = u.nblk - 1;
-    u.a1 = 0;
-    if (MODE != kLayoutSparse && u.row0 + 128 < u.len) {
-      const int hi0 = p.wr >= 0 ? min(u.len - 1, u.row0 + 127 + p.wr) : u.len - 1;
-      const int lo1 = p.wl >= 0 ? max(0, u.row0 + 128 - p.wl) : 0;
-      u.z0 = hi0 / 128 - u.first;
-      u.a1 = lo1 / 128 - u.first;
     }
   }
   return u;
@@ -471,28 +436,8 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
                     (acc || kk > 0) ? 1u : 0u);
         }
       };
-      // Barrier phases of the per-tile barriers (s_full, p_ready, s_read,
-      // p_free) count the blocks each query tile has visited: G0 / G1 at the
-      // start of the unit, so block it of tile t is number G_t + it - first.
-      int G0 = 0, G1 = 0;  // (two scalars: an array indexed by t would live in local memory)
-      auto blk = [&](const Unit& u, int t, int it) { return (t == 0 ? G0 : G1) + it - tile_first<MODE>(u, t); };
-      auto unit_done = [&](const Unit& u) {
-        G0 += tile_blocks<MODE>(u, 0);
-        G1 += tile_blocks<MODE>(u, 1);
-      };
-      // PV_t of relative block it (its V in slot sv), after the softmax has
-      // written P_t; the first PV of a tile in a unit overwrites O_t, which
-      // the previous unit's epilogue must have read.
-      auto pv_block = [&](const Unit& u, int k, int t, int it, int sv, int site) -> bool {
-        if (!wait_bar(p_ready(t), blk(u, t, it) & 1, ab, p.wait_ns, site)) return false;
-        if (it == tile_first<MODE>(u, t) && k > 0 && !wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7))
-          return false;
-        tc_fence_after();
-        pv(t, sv, it > tile_first<MODE>(u, t));
-        return true;
-      };
       if constexpr (DYN || C::PSEP) {
-        int n = 0;  // KV slots
+        int n = 0, g = 0;  // KV slots, blocks
         bool ok = true;
         for (int k = 0; ok; ++k) {
           int L;
@@ -512,11 +457,12 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
           ok = wait_bar(q_full(qb), (k >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
           if (!ok) break;
           if constexpr (C::PSEP) {
-            // Step it issues S_t of block it as soon as softmax t has read its
+            // Step it issues S_t of block it as soon as softmax t has read the
             // previous S_t, then PV_t of block it-1 once P_t is ready: each
             // softmax warpgroup finds its next S finished when it completes a
             // block.  K of block it sits in slot n + 2 it, V in the next one.
             for (int it = 0; it <= u.nblk && ok; ++it) {
+              const int gi = g + it;
               const int nk = n + 2 * it, nv = nk - 1;
               if (it < u.nblk) {
                 ok = wait_bar(slot_full(nk % SLOTS), (nk / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
@@ -527,19 +473,23 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
                 if (!ok) break;
               }
               for (int t = 0; t < NQT && ok; ++t) {
-                if (it < u.nblk && tile_needs<MODE>(u, t, it)) {
-                  const int gi = blk(u, t, it);
+                if (it < u.nblk) {
                   if (gi > 0) ok = wait_bar(s_read(t), (gi - 1) & 1, ab, p.wait_ns, SITE_MMA + 9);
                   if (!ok) break;
                   tc_fence_after();
                   qk(t, qb, nk % SLOTS);
                   umma_commit(s_full(t));
                 }
-                if (it > 0 && tile_needs<MODE>(u, t, it - 1)) {
-                  ok = pv_block(u, k, t, it - 1, nv % SLOTS, SITE_MMA + 3);
+                if (it > 0) {
+                  ok = wait_bar(p_ready(t), (gi - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
+                  // the first PV of a unit overwrites O_t: the previous unit's
+                  // epilogue must have read it
+                  if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
                   if (!ok) break;
+                  tc_fence_after();
+                  pv(t, nv % SLOTS, it > 1);
                   umma_commit(p_free(t));
-                  if (it == u.nblk || !tile_needs<MODE>(u, t, it)) umma_commit(o_full(t));
+                  if (it == u.nblk) umma_commit(o_full(t));
                 }
               }
               if (!ok) break;
@@ -551,7 +501,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             }
             if (!ok) break;
             n += 2 * u.nblk;
-            unit_done(u);
+            g += u.nblk;
             continue;
           }
           {
@@ -559,11 +509,10 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
             if (!ok) break;
             tc_fence_after();
-            for (int t = 0; t < NQT; ++t)
-              if (tile_needs<MODE>(u, t, 0)) {
-                qk(t, qb, sk);
-                umma_commit(s_full(t));
-              }
+            for (int t = 0; t < NQT; ++t) {
+              qk(t, qb, sk);
+              umma_commit(s_full(t));
+            }
             umma_commit(slot_empty(sk));
             if (u.nblk == 1) umma_commit(q_empty(qb));
             ++n;
@@ -572,20 +521,20 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             const int sv = n % SLOTS, sk = (n + 1) % SLOTS;
             ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
             for (int t = 0; t < NQT && ok; ++t) {
-              if (tile_needs<MODE>(u, t, it - 1)) {
-                ok = pv_block(u, k, t, it - 1, sv, SITE_MMA + 3);
-                if (!ok) break;
-                if (!tile_needs<MODE>(u, t, it)) umma_commit(o_full(t));  // tile 0 ended early
-              }
+              ok = wait_bar(p_ready(t), (g + it - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
+              // the first PV of a unit overwrites O_t: the previous unit's
+              // epilogue must have read it
+              if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+              if (!ok) break;
+              tc_fence_after();
+              pv(t, sv, it > 1);
               if (t == 0) {
                 ok = wait_bar(slot_full(sk), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 4);
                 if (!ok) break;
                 tc_fence_after();
               }
-              if (tile_needs<MODE>(u, t, it)) {
-                qk(t, qb, sk);
-                umma_commit(s_full(t));
-              }
+              qk(t, qb, sk);
+              umma_commit(s_full(t));
             }
             if (!ok) break;
             if (it == u.nblk - 1) umma_commit(q_empty(qb));  // the unit's last S products
@@ -598,15 +547,17 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             const int sv = n % SLOTS;
             ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 5);
             for (int t = 0; t < NQT && ok; ++t) {
-              if (!tile_needs<MODE>(u, t, u.nblk - 1)) continue;
-              ok = pv_block(u, k, t, u.nblk - 1, sv, SITE_MMA + 6);
+              ok = wait_bar(p_ready(t), (g + u.nblk - 1) & 1, ab, p.wait_ns, SITE_MMA + 6);
+              if (ok && u.nblk == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
               if (!ok) break;
+              tc_fence_after();
+              pv(t, sv, u.nblk > 1);
               umma_commit(o_full(t));
             }
             if (ok) umma_commit(slot_empty(sv));
             ++n;
           }
-          unit_done(u);
+          g += u.nblk;
         }
       } else {
         // Static schedule, P over S: the last block of a unit issues PV_t
@@ -619,7 +570,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
           const int L = unit_index(k);
           return L >= p.num_units ? -1 : L;
         };
-        int n = 0;  // KV slots
+        int n = 0, g = 0;  // KV slots, blocks
         bool ok = true;
         // this unit's first S products went out with the previous unit's last
         // PV products (every unit but the first)
@@ -635,11 +586,10 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
             if (!ok) break;
             tc_fence_after();
-            for (int t = 0; t < NQT; ++t)
-              if (tile_needs<MODE>(u, t, 0)) {
-                qk(t, qb, sk);
-                umma_commit(s_full(t));
-              }
+            for (int t = 0; t < NQT; ++t) {
+              qk(t, qb, sk);
+              umma_commit(s_full(t));
+            }
             umma_commit(slot_empty(sk));
             if (u.nblk == 1) umma_commit(q_empty(qb));
             ++n;
@@ -648,20 +598,20 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             const int sv = n % SLOTS, sk = (n + 1) % SLOTS;
             ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 2);
             for (int t = 0; t < NQT && ok; ++t) {
-              if (tile_needs<MODE>(u, t, it - 1)) {
-                ok = pv_block(u, k, t, it - 1, sv, SITE_MMA + 3);
-                if (!ok) break;
-                if (!tile_needs<MODE>(u, t, it)) umma_commit(o_full(t));  // tile 0 ended early
-              }
+              ok = wait_bar(p_ready(t), (g + it - 1) & 1, ab, p.wait_ns, SITE_MMA + 3);
+              // the first PV of a unit overwrites O_t: the previous unit's
+              // epilogue must have read it
+              if (ok && it == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+              if (!ok) break;
+              tc_fence_after();
+              pv(t, sv, it > 1);
               if (t == 0) {
                 ok = wait_bar(slot_full(sk), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 4);
                 if (!ok) break;
                 tc_fence_after();
               }
-              if (tile_needs<MODE>(u, t, it)) {
-                qk(t, qb, sk);
-                umma_commit(s_full(t));
-              }
+              qk(t, qb, sk);
+              umma_commit(s_full(t));
             }
             if (!ok) break;
             if (it == u.nblk - 1) umma_commit(q_empty(qb));  // the unit's last S products
@@ -676,11 +626,12 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             Unit un{};
             ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 5);
             for (int t = 0; t < NQT && ok; ++t) {
-              if (tile_needs<MODE>(u, t, u.nblk - 1)) {
-                ok = pv_block(u, k, t, u.nblk - 1, sv, SITE_MMA + 6);
-                if (!ok) break;
-                umma_commit(o_full(t));
-              }
+              ok = wait_bar(p_ready(t), (g + u.nblk - 1) & 1, ab, p.wait_ns, SITE_MMA + 6);
+              if (ok && u.nblk == 1 && k > 0) ok = wait_bar(o_empty(t), (k - 1) & 1, ab, p.wait_ns, SITE_MMA + 7);
+              if (!ok) break;
+              tc_fence_after();
+              pv(t, sv, u.nblk > 1);
+              umma_commit(o_full(t));
               if (t == 0) {
                 Ln = fetch(k + 1);
                 if (Ln >= 0) {
@@ -691,7 +642,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
                 }
                 if (!ok) break;
               }
-              if (Ln >= 0 && tile_needs<MODE>(un, t, 0)) {
+              if (Ln >= 0) {
                 qk(t, qbn, skn);
                 umma_commit(s_full(t));
               }
@@ -707,7 +658,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             L = Ln;
             s0_issued = true;
           }
-          unit_done(u);
+          g += u.nblk;
         }
       }
       // Drain: wait until every MMA issued above has completed.
@@ -815,17 +766,13 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
       float slope2 = 0.f;
       if (ALIBI) slope2 = -p.alibi[h] * LOG2E;
       float m_run = -CUDART_INF_F, l_run = 0.f;
-      // this tile's blocks of the unit: [it0, it0 + nbt) (all of them with a
-      // block mask, which hides blocks element-wise instead)
-      const int it0 = tile_first<MODE>(u, t), nbt = tile_blocks<MODE>(u, t);
       int kb = u.first;
-      for (int it = it0; it < it0 + nbt; ++it, kb = next_block<MODE>(p, u, kb)) {
+      for (int it = 0; it < u.nblk; ++it, kb = next_block<MODE>(p, u, kb)) {
         const int kv0 = (SPARSE ? kb : u.first + it) * BN;
-        const int gi = g + it - it0;  // this tile's block count: barrier phases
         // block hidden from this tile by the block mask (it is visited for
         // the other tile of the pair, or to write a fully hidden unit)
         const bool hidden = SPARSE && (mrow == nullptr || mrow[kb] == 0);
-        ok = wait_bar(s_full(t), gi & 1, ab, p.wait_ns, SITE_SOFT + 0);
+        ok = wait_bar(s_full(t), (g + it) & 1, ab, p.wait_ns, SITE_SOFT + 0);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
@@ -890,9 +837,9 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         upk2(add2(l2x[0], l2x[1]), la, lb);
         upk2(add2(l2x[2], l2x[3]), lc, ld);
         l_run = fmaf(l_run, alpha, (la + lb) + (lc + ld));
-        if (C::PSEP && gi > 0) {
+        if (C::PSEP && g + it > 0) {
           // P_t and O_t are free once the previous block's PV product is done
-          ok = wait_bar(p_free(t), (gi - 1) & 1, ab, p.wait_ns, SITE_SOFT + 6);
+          ok = wait_bar(p_free(t), (g + it - 1) & 1, ab, p.wait_ns, SITE_SOFT + 6);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
@@ -937,7 +884,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         // Rescale the running output (the PV product of the previous block has
         // completed: S_t of this block was committed after it, or, with the
         // separate-P layout, p_free said so).
-        if (it > it0 && __any_sync(0xffffffffu, resc)) {
+        if (it > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
             uint32_t w32[32];
@@ -954,7 +901,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         // first unit, whichever schedule) withholds tile 0's arrive on the
         // first block, so the MMA warp's bounded wait for it runs out and
         // every role of that CTA winds down through the abort path.
-        if (!(p.test_skip && L == 0 && it == it0 && t == 0)) bar_arrive(p_ready(t));
+        if (!(p.test_skip && L == 0 && it == 0 && t == 0)) bar_arrive(p_ready(t));
       }
       if (!ok) break;
       // ------------------------------------ hand the row's results over
@@ -966,7 +913,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
       stats[t * BM + r] = make_float2(l_run > 0.f ? 1.f / l_run : 0.f,
                                       l_run > 0.f ? (m_run + log2f(l_run)) * LN2 : -CUDART_INF_F);
       bar_arrive(stats_full(t));
-      g += nbt;
+      g += u.nblk;
     }
   }
 

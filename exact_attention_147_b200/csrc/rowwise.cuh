@@ -1,6 +1,7 @@
 // Memory-bound row kernels of the backward pass:
 //   bwd_preprocess : D[b,h,i] = sum_c dO[b,i,h,c] * O[b,i,h,c]   (fp32)
-//   dq_convert     : dQ[b,i,h,:] = scale * dQaccum[b,h,i,:] cast to bf16
+//   dq_convert     : dQ[b,i,h,:] = scale * dQaccum[b,h,i,:] cast to bf16 (or
+//                    the sum of two accumulators, in a fixed order)
 // Each row of d elements is read by a group of lanes with 16-byte vector
 // loads (d * element size / 16 lanes per row), so every warp touches whole
 // 32-byte sectors; rows are ordered with i fastest so the fp32 [B,H,N]
@@ -63,8 +64,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const AttnArgs a) {
   if (R < rows && li == 0) const_cast<float*>(a.dvec)[R] = s;
 }
 
-// dQaccum (fp32, [B,H,N,d] dense) -> dQ (bf16, strided [B,N,H,d]).
-template <int HD>
+// dQaccum (fp32, [B,H,N,d] dense) -> dQ (bf16, strided [B,N,H,d]).  With
+// NACC = 2 the workspace holds two such accumulators back to back (the
+// ordered deterministic backward's even and odd key blocks), added here in
+// that fixed order.
+template <int HD, int NACC = 1>
 __global__ void __launch_bounds__(256) dq_convert_kernel(const AttnArgs a) {
   constexpr int L = HD / 4;  // lanes per row, 4 floats each
   const long long rows = (long long)a.B * a.H * a.N;
@@ -74,7 +78,11 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const AttnArgs a) {
   const int n = int(R % a.N);
   const long long bh = R / a.N;
   const int h = int(bh % a.H), b = int(bh / a.H);
-  const float4 v = *reinterpret_cast<const float4*>(a.dq_accum + R * HD + li * 4);
+  float4 v = *reinterpret_cast<const float4*>(a.dq_accum + R * HD + li * 4);
+  if (NACC == 2) {
+    const float4 w2 = *reinterpret_cast<const float4*>(a.dq_accum + (rows + R) * HD + li * 4);
+    v = make_float4(v.x + w2.x, v.y + w2.y, v.z + w2.z, v.w + w2.w);
+  }
   __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(a.dq) + b * a.sdq.b + (long long)n * a.sdq.n +
                       h * a.sdq.h + li * 4;
   __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * a.scale, v.y * a.scale);

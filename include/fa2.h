@@ -168,8 +168,9 @@ fa2_status fa2_bwd_preprocess(const void* o, const void* dout, float* D,
 
 /*
  * Bytes of device workspace fa2_bwd needs for these shapes: for bf16, an fp32
- * dQ accumulator (B * H * N * d floats) and, when deterministic, one 32-bit
- * counter per 32 query rows (B * H * ceil(N / 128) * 4); nothing for fp32.
+ * dQ accumulator (B * H * N * d floats) -- when deterministic, two of them
+ * and, for each, one 32-bit counter per 32 query rows
+ * (B * H * ceil(N / 128) * 4); nothing for fp32.
  * The caller allocates it; its contents on entry do not matter (the call
  * clears what it uses).  Returns 0 for invalid shapes.
  */
@@ -204,9 +205,11 @@ size_t fa2_bwd_workspace_size(int B, int N, int H, int d, fa2_dtype dtype, int d
  *                    (fast, bits may differ between runs);
  *                    nonzero: dq, dk and dv are bitwise repeatable.  Under a
  *                    causal mask (window_right = 0) the partial sums of each
- *                    query block are added in a fixed order (descending key
- *                    block) inside the same kernel; otherwise dQ comes from
- *                    a second, ordered pass that recomputes the scores.
+ *                    query block are added in a fixed order inside the same
+ *                    kernel (even and odd key blocks into two accumulators,
+ *                    each in descending key-block order, then the two added);
+ *                    otherwise dQ comes from a second, ordered pass that
+ *                    recomputes the scores.
  */
 fa2_status fa2_bwd(const void* q, const void* k, const void* v, const void* dout,
                    const float* lse, const float* D, void* dq, void* dk, void* dv,

@@ -15,7 +15,7 @@ from exact_attention_147_b200 import fa2 as F
 from exact_attention_147_b200 import workloads as W
 from oracle import attention as oa
 from oracle import philox
-from tests.helpers import check_fwd, check_grad, d_rounding_bounds, f64
+from tests.helpers import assert_same_sum_any_order, check_fwd, check_grad, d_rounding_bounds, f64
 
 pytestmark = pytest.mark.gpu
 
