@@ -882,9 +882,16 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
             // last first, so a box only ever waits for items taken earlier
             // (no wait can close a cycle).  A counter per box and accumulator
             // holds how many sums it has received: wait for our rank, add, and
-            // raise it once the adds are complete, which is checked after the
-            // next box's adds have been issued (or at the end of the item),
-            // so the drain keeps one box's adds in flight.
+            // raise it once the adds are complete.  That is checked at the
+            // next box, before its own turn is awaited: a release must never
+            // wait behind a later box's turn, or the waits of one chain would
+            // queue behind those of the chains further down the diagonal.
+            if (lane == 0 && pend_box >= 0) {
+              bulk_wait_all();  // the previous box's adds are complete
+              fence_proxy_async_global();
+              st_release_gpu(p.dq_chain + pend_box, pend_val);
+            }
+            pend_box = -1;
             const int acc = itm.kb & 1;
             const long long box =
                 ((long long)(acc * p.B * p.H + bh) * p.nblocks + qb) * 4 + wq;
@@ -898,11 +905,6 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
             if (!ok) break;
 #pragma unroll
             for (int c = 0; c < NC; ++c) stage(u[c], c, acc);
-            if (lane == 0 && pend_box >= 0) {
-              bulk_wait_upto<NC>();  // the previous box's adds are complete
-              fence_proxy_async_global();
-              st_release_gpu(p.dq_chain + pend_box, pend_val);
-            }
             pend_box = box;
             pend_val = rank + 1u;
             continue;
