@@ -76,6 +76,10 @@ DropoutParams make_dropout(float dropout_p, unsigned long long seed) {
   d.seed_hi = uint32_t(seed >> 32);
   d.threshold = uint32_t(t);
   d.keep_scale = float(256.0 / (256.0 - t));
+  for (int r = 0; r < kPhiloxRounds; ++r) {  // Philox4x32's Weyl key schedule
+    d.rk0[r] = d.seed_lo + uint32_t(r) * 0x9E3779B9u;
+    d.rk1[r] = d.seed_hi + uint32_t(r) * 0xBB67AE85u;
+  }
   return d;
 }
 

@@ -21,27 +21,31 @@
 
 namespace fa2 {
 
+constexpr int kPhiloxRounds = 10;
+
 struct DropoutParams {
   uint32_t seed_lo, seed_hi;
   uint32_t threshold;   // t in [0, 255]
   float keep_scale;     // 256 / (256 - t)
+  // The key of round r, (seed_lo + r 0x9E3779B9, seed_hi + r 0xBB67AE85) mod
+  // 2^32: the same for every generator call of a launch, so it is formed
+  // once on the host, and the rounds read it from the kernel's parameters.
+  uint32_t rk0[kPhiloxRounds], rk1[kPhiloxRounds];
 };
 
 struct Philox4 {
   uint32_t w[4];
 };
 
+// One 32 x 32 -> 64-bit product gives both halves a round needs.
 __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
-                                                 uint32_t k0, uint32_t k1) {
+                                                 const DropoutParams& dp) {
 #pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    if (r > 0) {
-      k0 += 0x9E3779B9u;
-      k1 += 0xBB67AE85u;
-    }
-    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
-    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
-    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+  for (int r = 0; r < kPhiloxRounds; ++r) {
+    const uint64_t p0 = uint64_t(0xD2511F53u) * c0, p1 = uint64_t(0xCD9E8D57u) * c2;
+    const uint32_t lo0 = uint32_t(p0), hi0 = uint32_t(p0 >> 32);
+    const uint32_t lo1 = uint32_t(p1), hi1 = uint32_t(p1 >> 32);
+    const uint32_t n0 = hi1 ^ c1 ^ dp.rk0[r], n2 = hi0 ^ c3 ^ dp.rk1[r];
     c0 = n0;
     c1 = lo1;
     c2 = n2;
@@ -57,8 +61,7 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
 
 // Four random bytes (keys 4*j4 .. 4*j4+3) of query row i, packed in a word.
 __device__ __forceinline__ uint32_t dropout_word_row(const DropoutParams& dp, int b, int h, int i, int j4) {
-  const Philox4 o = philox4x32_10(uint32_t(j4), uint32_t(i >> 2), uint32_t(h), uint32_t(b), dp.seed_lo,
-                                  dp.seed_hi);
+  const Philox4 o = philox4x32_10(uint32_t(j4), uint32_t(i >> 2), uint32_t(h), uint32_t(b), dp);
   const int s = i & 3;
   return s == 0 ? o.w[0] : s == 1 ? o.w[1] : s == 2 ? o.w[2] : o.w[3];
 }
@@ -99,8 +102,7 @@ __device__ __forceinline__ void quad_transpose(const uint32_t (&x)[4], uint32_t 
 __device__ __forceinline__ void dropout_words_row16(const DropoutParams& dp, int b, int h, int i, int j4_0,
                                                     uint32_t (&z)[4]) {
   const int s = int(threadIdx.x & 3u);
-  const Philox4 o = philox4x32_10(uint32_t(j4_0 + s), uint32_t(i >> 2), uint32_t(h), uint32_t(b),
-                                  dp.seed_lo, dp.seed_hi);
+  const Philox4 o = philox4x32_10(uint32_t(j4_0 + s), uint32_t(i >> 2), uint32_t(h), uint32_t(b), dp);
   // word w of call (j4_0 + s) belongs to row 4 (i / 4) + w, i.e. quad lane w
   quad_transpose(o.w, z);
 }
@@ -112,8 +114,7 @@ __device__ __forceinline__ void dropout_words_row16(const DropoutParams& dp, int
 __device__ __forceinline__ void dropout_words_col16(const DropoutParams& dp, int b, int h, int j, int i4_0,
                                                     uint32_t (&z)[4]) {
   const int s = int(threadIdx.x & 3u);
-  const Philox4 o = philox4x32_10(uint32_t(j >> 2), uint32_t(i4_0 + s), uint32_t(h), uint32_t(b),
-                                  dp.seed_lo, dp.seed_hi);
+  const Philox4 o = philox4x32_10(uint32_t(j >> 2), uint32_t(i4_0 + s), uint32_t(h), uint32_t(b), dp);
   // byte r of every word belongs to key 4 (j / 4) + r, i.e. quad lane r:
   // transpose the 4 x 4 bytes so that x[r] gathers byte r of words 0..3
   const uint32_t lo01 = __byte_perm(o.w[0], o.w[1], 0x5140), hi01 = __byte_perm(o.w[0], o.w[1], 0x7362);
