@@ -99,3 +99,47 @@ def test_more_streams_than_counter_pairs():
         torch.cuda.synchronize()
         for hnd in handles:
             rt.cudaStreamDestroy(hnd)
+
+
+def test_counter_calls_inside_a_cuda_graph():
+    # A counter-scheduled call captured into a CUDA graph keeps the pair of
+    # its capturing stream; the pair is cleared by a captured memset before
+    # the kernel, so the graph replays correctly any number of times.  The
+    # first call on the stream is made before the capture (it may take the
+    # pair over from another stream, which needs an event wait that a capture
+    # cannot record).
+    q, k, v, do = W.make_inputs(SHORT, "cuda")
+    cu = SHORT.cu_seqlens("cuda")
+    ref_o, ref_l = F.fwd_varlen(q, k, v, cu, SHORT.N, causal=True)
+    ref_D = F.bwd_preprocess(ref_o, do)
+    ref_g = F.bwd_varlen(do, q, k, v, ref_l, ref_D, cu, SHORT.N, causal=True, deterministic=True)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    out, lse = torch.empty_like(ref_o), torch.empty_like(ref_l)
+    D = torch.empty_like(ref_D)
+    g = [torch.empty_like(t) for t in ref_g]
+    ws = torch.empty(max(1, F.workspace_size(1, SHORT.total, SHORT.H, SHORT.d, torch.bfloat16, True)),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        F.fwd_varlen(q, k, v, cu, SHORT.N, causal=True, out=out, lse=lse, stream=s)
+        F.bwd_preprocess(out, do, D, stream=s)
+        F.bwd_varlen(do, q, k, v, lse, D, cu, SHORT.N, causal=True, deterministic=True, dq=g[0],
+                     dk=g[1], dv=g[2], workspace=ws, stream=s)
+
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()                       # outside the capture: the stream takes its pair
+    s.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        step()
+    for _ in range(2):
+        for t in (out, lse, *g):
+            t.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert F.device_status() == 0
+        assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+        assert all(torch.equal(a, b) for a, b in zip(g, ref_g))
+    del graph

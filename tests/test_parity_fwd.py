@@ -113,6 +113,16 @@ def test_long_local_sampled():
     sampled_compare(w, [(0, 0)], n_rows=64)
 
 
+@pytest.mark.parametrize("d,causal", [(128, False), (128, True), (64, True)])
+def test_very_long_sequence_sampled(d, causal):
+    # one head of 262144 tokens (2048 key blocks, 1024 units): unit counts,
+    # TMA row coordinates and the statistics index reach far beyond the
+    # workloads' sizes; sampled rows against the oracle
+    w = W.Workload(f"long-{d}{'-causal' if causal else ''}", B=1, N=262144, H=1, d=d,
+                   causal=causal, seed=140 + d)
+    sampled_compare(w, [], n_rows=24)
+
+
 def test_alibi_sampled():
     w = W.alibi_det()
     sampled_compare(w, [(1, 5)], n_rows=16)
