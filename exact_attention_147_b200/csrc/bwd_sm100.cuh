@@ -724,12 +724,16 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = c * 32 + 2 * e;
-            float a0 = pr[c0], a1 = pr[c0 + 1];
             if (DROPOUT) {
-              a0 = kept(c0) ? a0 * p.drop.keep_scale : 0.f;
-              a1 = kept(c0 + 1) ? a1 * p.drop.keep_scale : 0.f;
+              // the pair's two keep bits become 0xFFFF over each kept bf16
+              // half: ((bits 0x8001) & 0x10001) 0xFFFF maps 0,1,2,3 to
+              // 0, 0xFFFF, 0xFFFF0000, 0xFFFFFFFF (a dropped half is +0)
+              const uint32_t two = ((c == 0 ? keep_lo : keep_hi) >> (2 * e)) & 3u;
+              w[e] = pack_bf16(pr[c0] * p.drop.keep_scale, pr[c0 + 1] * p.drop.keep_scale) &
+                     (((two * 0x8001u) & 0x10001u) * 0xFFFFu);
+            } else {
+              w[e] = pack_bf16(pr[c0], pr[c0 + 1]);
             }
-            w[e] = pack_bf16(a0, a1);
           }
           tmem_st16(tmem + lane_base + T_S + cq + c * 16, w);
         }
