@@ -254,8 +254,10 @@ fa2_status launched(int n) {
 // each launch (the call's last CTA clears it too), which also repairs a pair
 // that an aborted call left non-zero.  Up to kSchedSlots streams per device
 // own a pair at a time; a further stream takes over the pair used least
-// recently, after making itself wait (cudaStreamWaitEvent) for the event
-// recorded after that pair's last launch, so the two calls cannot overlap.
+// recently.  Every launch (outside stream capture) first makes its stream
+// wait (cudaStreamWaitEvent) for the event recorded after the pair's last
+// launch, so two calls can never overlap on a pair -- also when a stream
+// handle is destroyed and reused while its last call still runs.
 // During stream capture nothing is recorded: the captured call keeps the
 // capturing stream's pair, and a hand-over that would need a wait is refused
 // (FA2_ERR_UNSUPPORTED).
@@ -287,13 +289,21 @@ class SchedLease {
       if (t.owned[i] && t.owner[i] == st) s = i;
     for (int i = 0; i < kSchedSlots && s < 0; ++i)
       if (!t.owned[i]) s = i;
+    bool handover = false;
     if (s < 0) {  // every pair is owned: take over the least recently used one
       s = 0;
       for (int i = 1; i < kSchedSlots; ++i)
         if (t.last_use[i] < t.last_use[s]) s = i;
-      if (t.done_valid[s]) {
-        if (capturing_) return FA2_ERR_UNSUPPORTED;
-        if (cudaStreamWaitEvent(st, t.done[s], 0) != cudaSuccess) return FA2_ERR_CUDA;
+      handover = true;
+    }
+    // Order this launch after the pair's last one.  On the pair's own stream
+    // that costs nothing on the GPU, and it keeps the pair safe when a stream
+    // handle is destroyed and handed out again while its last call still runs.
+    if (t.done_valid[s]) {
+      if (capturing_) {
+        if (handover) return FA2_ERR_UNSUPPORTED;  // a capture cannot wait on it
+      } else if (cudaStreamWaitEvent(st, t.done[s], 0) != cudaSuccess) {
+        return FA2_ERR_CUDA;
       }
     }
     if (!capturing_ && t.done[s] == nullptr &&

@@ -46,9 +46,12 @@
  *    stream that makes such calls owns one pair: calls on one stream run in
  *    order and reuse it, calls on different streams never share one while
  *    both may run.  The pair is cleared on the call's stream before each
- *    launch.  Up to 64 streams per device own a pair at a time; a further
- *    stream takes over the least recently used pair after waiting, on the
- *    GPU (an event), for that pair's last call to finish.  During stream
+ *    launch, after the stream has been made to wait, on the GPU (an
+ *    event), for the pair's last call to finish (free on the pair's own
+ *    stream; it also covers a stream handle that is destroyed and reused
+ *    while its last call still runs).  Up to 64 streams per device own a
+ *    pair at a time; a further stream takes over the least recently used
+ *    pair behind the same wait.  During stream
  *    capture no such wait can be recorded: a captured call keeps the pair
  *    of the capturing stream (a hand-over that would need a wait returns
  *    FA2_ERR_UNSUPPORTED), and the caller must not replay the graph while

@@ -143,3 +143,32 @@ def test_counter_calls_inside_a_cuda_graph():
         assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
         assert all(torch.equal(a, b) for a, b in zip(g, ref_g))
     del graph
+
+
+def test_stream_destroyed_while_its_call_runs():
+    # The long call's stream is destroyed right after the launch; a new
+    # stream (which may be handed the same handle) makes a short call at
+    # once.  Each launch waits for the event of its pair's previous launch, so
+    # the two cannot split one counter whether or not the handle is reused.
+    ql, kl, vl, cul = _fwd_inputs(LONG)
+    qs, ks, vs, cus = _fwd_inputs(SHORT)
+    ref_long = F.fwd_varlen(ql, kl, vl, cul, LONG.N, causal=LONG.causal)
+    ref_short = F.fwd_varlen(qs, ks, vs, cus, SHORT.N, causal=SHORT.causal)
+    out_l, lse_l = torch.empty_like(ref_long[0]), torch.empty_like(ref_long[1])
+    out_s, lse_s = torch.empty_like(ref_short[0]), torch.empty_like(ref_short[1])
+    torch.cuda.synchronize()
+    (h1,) = _new_streams(1)
+    F.fwd_varlen(ql, kl, vl, cul, LONG.N, causal=LONG.causal, out=out_l, lse=lse_l,
+                 stream=torch.cuda.ExternalStream(h1))
+    rt.cudaStreamDestroy(h1)
+    (h2,) = _new_streams(1)
+    try:
+        F.fwd_varlen(qs, ks, vs, cus, SHORT.N, causal=SHORT.causal, out=out_s, lse=lse_s,
+                     stream=torch.cuda.ExternalStream(h2))
+        torch.cuda.synchronize()
+        assert F.device_status() == 0
+        assert torch.equal(out_l, ref_long[0]) and torch.equal(lse_l, ref_long[1])
+        assert torch.equal(out_s, ref_short[0]) and torch.equal(lse_s, ref_short[1])
+    finally:
+        torch.cuda.synchronize()
+        rt.cudaStreamDestroy(h2)
