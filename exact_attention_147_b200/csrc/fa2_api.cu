@@ -394,7 +394,8 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   SchedLease lease;
   if (MODE != kLayoutPadded) FA2_TRY(lease.acquire(dev, device_info(dev), st, &p.sched));
   auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, MODE, FP8>;
-  constexpr int smem = FwdCfg<HD, FP8>::SMEM_BYTES;
+  using Cfg = FwdCfg<HD, FP8, DROPOUT && HD == 128>;  // the kernel's own configuration
+  constexpr int smem = Cfg::SMEM_BYTES;
   FA2_TRY(ensure_smem(kern, smem, dev, mask));
   // The kernel re-balances registers between its warpgroups; the shares add
   // up to 512 threads x REGS_AT_LAUNCH, so it must launch with that many per
@@ -402,11 +403,11 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return FA2_ERR_CUDA;
-    if (fa.numRegs < FwdCfg<HD, FP8>::REGS_AT_LAUNCH) return FA2_ERR_UNSUPPORTED;
+    if (fa.numRegs < Cfg::REGS_AT_LAUNCH) return FA2_ERR_UNSUPPORTED;
   }
   // persistent grid: one CTA per SM (shared memory and TMEM allow one)
   const unsigned grid = unsigned(std::min(p.num_units, std::max(sm_count, 1)));
-  kern<<<grid, FwdCfg<HD, FP8>::THREADS, smem, st>>>(p);
+  kern<<<grid, Cfg::THREADS, smem, st>>>(p);
   FA2_TRY(launched(1));
   return lease.finish();
 }

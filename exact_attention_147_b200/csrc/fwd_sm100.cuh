@@ -94,27 +94,33 @@ struct FwdParams {
   int test_skip;                       // test switch, 0 in normal use: see the softmax's p_ready arrive
 };
 
-template <int HD, bool FP8 = false>
+template <int HD, bool FP8 = false, bool MASK_EPI = false>
 struct FwdCfg {
   static constexpr int BM = 128;        // query rows per tile
   static constexpr int BN = 128;        // keys per KV block
   static constexpr int NQT = 2;         // query tiles per unit
-  static constexpr int QBUFS = 2;       // Q double buffer (across units)
+  // MASK_EPI (d = 128 with dropout): the epilogue warps draw each block's
+  // dropout mask into shared memory ahead of the softmax, in a ring of
+  // MASK_RING blocks of keep bytes; Q is single-buffered to make room.
+  static constexpr int QBUFS = MASK_EPI ? 1 : 2;  // Q buffers (across units)
   static constexpr int ESZ = FP8 ? 1 : 2;                    // bytes per element
   static constexpr int KSTEP = FP8 ? 32 : 16;                // K of one MMA
   static constexpr int SLOTS = FP8 ? 6 : (HD == 128 ? 3 : 8);
   static constexpr int QT_BYTES = BM * HD * ESZ;
   static constexpr int KV_BYTES = BN * HD * ESZ;
   static constexpr int OFF_KV = QBUFS * NQT * QT_BYTES;
-  static constexpr int OFF_BARS = OFF_KV + SLOTS * KV_BYTES;
+  static constexpr int MASK_RING = 2;
+  static constexpr int MASK_BYTES = NQT * BM * BN;  // one block's keep bytes, both tiles
+  static constexpr int OFF_MASK = OFF_KV + SLOTS * KV_BYTES;
+  static constexpr int OFF_BARS = OFF_MASK + (MASK_EPI ? MASK_RING * MASK_BYTES : 0);
   static constexpr int RING = 4;        // unit-index ring of the packed scheduler
   // d = 64 leaves 128 TMEM columns free: P gets its own 64 columns per tile,
   // so the next S product need not wait for the PV product that reads P.
   static constexpr bool PSEP = HD == 64 && !FP8;
   // q_full[2], q_empty[2], slot full/empty, s_full[2], p_ready[2], o_full[2],
   // o_empty[2], drain, ring full[4], ring empty[4], stats_full[2], stats_free[2],
-  // s_read[2], p_free[2]
-  static constexpr int NBARS = 2 * QBUFS + 2 * SLOTS + 4 * NQT + 1 + 2 * RING + 4 * NQT;
+  // s_read[2], p_free[2], mask_full[MASK_RING], mask_empty[MASK_RING]
+  static constexpr int NBARS = 4 + 2 * SLOTS + 4 * NQT + 1 + 2 * RING + 4 * NQT + (MASK_EPI ? 2 * MASK_RING : 0);
   // barriers, then the TMEM address, the abort flag, 2 spare words, the ring
   // and the per-row results (1 / l, LSE) the softmax hands to the epilogue
   static constexpr int OFF_STATS = OFF_BARS + NBARS * 8 + 16 + 4 * RING;
@@ -267,9 +273,12 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 
 template <int HD, bool ALIBI, bool DROPOUT, int MODE, bool FP8 = false>
 __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<HD, FP8>;
+  // d = 128 with dropout: the epilogue warps draw the mask (see FwdCfg)
+  constexpr bool MASK_EPI = DROPOUT && HD == 128;
+  using C = FwdCfg<HD, FP8, MASK_EPI>;
   static_assert(!FP8 || (HD == 128 && !DROPOUT && MODE == kLayoutPadded),
                 "e4m3 inputs: d = 128, padded layout, no dropout");
+  constexpr int QBUFS = C::QBUFS;
   constexpr bool PACKED = MODE == kLayoutPacked;
   constexpr bool SPARSE = MODE == kLayoutSparse;
   constexpr bool DYN = PACKED || SPARSE;  // units taken from the shared counter
@@ -309,6 +318,11 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
   // separate-P layout only: S_t has been read into registers / P_t has been read by its PV product
   auto s_read = [&](int t) { return bar0 + 8u * (17 + 2 * SLOTS + 2 * C::RING + t); };
   auto p_free = [&](int t) { return bar0 + 8u * (19 + 2 * SLOTS + 2 * C::RING + t); };
+  // MASK_EPI: a block's keep bytes written by the epilogue / read by both softmax warpgroups
+  auto mask_full = [&](int m) { return bar0 + 8u * (21 + 2 * SLOTS + 2 * C::RING + m); };
+  auto mask_empty = [&](int m) { return bar0 + 8u * (21 + 2 * SLOTS + 2 * C::RING + C::MASK_RING + m); };
+  // [MASK_RING][NQT][BN / 16][BM] x 16 keep bytes (keys 16 c .. 16 c + 15 of one row)
+  uint4* sMask = reinterpret_cast<uint4*>(smem_raw + C::OFF_MASK);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* ring = abort_flag + 3;  // packed: unit indices handed from the producer to the other roles
@@ -326,6 +340,12 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
       if (bar == stats_full(0) || bar == stats_full(1) || bar == stats_free(0) || bar == stats_free(1))
         cnt = 128;
       if (bar == s_read(0) || bar == s_read(1)) cnt = 128;
+      if (MASK_EPI) {
+        for (int m = 0; m < C::MASK_RING; ++m) {
+          if (bar == mask_full(m)) cnt = 128;   // the epilogue threads
+          if (bar == mask_empty(m)) cnt = 256;  // the softmax threads of both tiles
+        }
+      }
       // MMA + 8 softmax warps + 4 epilogue warps
       if (bar >= ring_empty(0) && bar <= ring_empty(C::RING - 1)) cnt = 13;
       bar_init(bar, cnt);
@@ -366,8 +386,8 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         }
         const Unit u = unit_of<MODE>(p, L);
         const int L_next = DYN ? fetch_unit<MODE>(p) : unit_index(k + 1);
-        const int qb = k & 1;
-        if (!wait_bar(q_empty(qb), ((k >> 1) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + 2)) break;
+        const int qb = k % QBUFS;
+        if (!wait_bar(q_empty(qb), ((k / QBUFS) & 1) ^ 1, ab, p.wait_ns, SITE_PROD + 2)) break;
         bar_arrive_expect_tx(q_full(qb), NQT * C::QT_BYTES);
         for (int t = 0; t < NQT; ++t)
           for (int c = 0; c < NCH; ++c)
@@ -396,7 +416,8 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
       // The last CTA to finish taking units returns the counters to zero.
       if (DYN) sched_cta_done(p.sched);
       // Before the CTA may exit, every copy issued must have landed.
-      for (int j = max(0, q_issued - 2); j < q_issued; ++j) drain_wait(q_full(j & 1), (j >> 1) & 1, p.wait_ns);
+      for (int j = max(0, q_issued - QBUFS); j < q_issued; ++j)
+        drain_wait(q_full(j % QBUFS), (j / QBUFS) & 1, p.wait_ns);
       for (int j = (n > SLOTS ? n - SLOTS : 0); j < n; ++j)
         drain_wait(slot_full(j % SLOTS), (j / SLOTS) & 1, p.wait_ns);
     }
@@ -453,8 +474,8 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
             if (L >= p.num_units) break;
           }
           const Unit u = unit_of<MODE>(p, L);
-          const int qb = k & 1;
-          ok = wait_bar(q_full(qb), (k >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
+          const int qb = k % QBUFS;
+          ok = wait_bar(q_full(qb), (k / QBUFS) & 1, ab, p.wait_ns, SITE_MMA + 0);
           if (!ok) break;
           if constexpr (C::PSEP) {
             // Step it issues S_t of block it as soon as softmax t has read the
@@ -578,9 +599,9 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         int L = fetch(0);
         for (int k = 0; ok && L >= 0; ++k) {
           const Unit u = unit_of<MODE>(p, L);
-          const int qb = k & 1;
+          const int qb = k % QBUFS;
           if (!s0_issued) {
-            ok = wait_bar(q_full(qb), (k >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
+            ok = wait_bar(q_full(qb), (k / QBUFS) & 1, ab, p.wait_ns, SITE_MMA + 0);
             if (!ok) break;
             const int sk = n % SLOTS;
             ok = wait_bar(slot_full(sk), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
@@ -621,7 +642,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
           }
           if (!ok) break;
           {  // last block, with the next unit's first S products
-            const int sv = n % SLOTS, skn = (n + 1) % SLOTS, qbn = (k + 1) & 1;
+            const int sv = n % SLOTS, skn = (n + 1) % SLOTS, qbn = (k + 1) % QBUFS;
             int Ln = -1;
             Unit un{};
             ok = wait_bar(slot_full(sv), (n / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 5);
@@ -636,7 +657,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
                 Ln = fetch(k + 1);
                 if (Ln >= 0) {
                   un = unit_of<MODE>(p, Ln);
-                  ok = wait_bar(q_full(qbn), ((k + 1) >> 1) & 1, ab, p.wait_ns, SITE_MMA + 0);
+                  ok = wait_bar(q_full(qbn), ((k + 1) / QBUFS) & 1, ab, p.wait_ns, SITE_MMA + 0);
                   if (ok) ok = wait_bar(slot_full(skn), ((n + 1) / SLOTS) & 1, ab, p.wait_ns, SITE_MMA + 1);
                   if (ok) tc_fence_after();
                 }
@@ -677,32 +698,19 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
     const uint32_t lane_base = uint32_t((warp % 4) * 32) << 16;
     const float o_mult = DROPOUT ? p.drop.keep_scale : (FP8 ? p.o_scale : 1.f);
     bool ok = true;
-    for (int k = 0; ok; ++k) {
-      int L;
-      if (DYN) {
-        const int rr = k % C::RING;
-        ok = wait_bar(ring_full(rr), (k / C::RING) & 1, ab, p.wait_ns, SITE_SOFT + 3);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        L = ring[rr];
-        __syncwarp();
-        if (lane == 0) bar_arrive(ring_empty(rr));
-        if (L < 0) break;
-      } else {
-        L = unit_index(k);
-        if (L >= p.num_units) break;
-      }
-      const Unit u = unit_of<MODE>(p, L);
+    // the output rows of unit u (the k-th unit of this CTA)
+    auto store_unit = [&](const Unit& u, int k) -> bool {
       const SeqView sv = PACKED ? seq_view(p.cu_seqlens, u.b, p.N, p.total) : SeqView{u.b, 0, p.N};
-      for (int t = 0; t < NQT && ok; ++t) {
+      for (int t = 0; t < NQT; ++t) {
         const int i = u.row0 + t * BM + r;  // local query row (>= len for padding rows)
-        ok = wait_bar(stats_full(t), k & 1, ab, p.wait_ns, SITE_SOFT + 4);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
+        bool okt = wait_bar(stats_full(t), k & 1, ab, p.wait_ns, SITE_SOFT + 4);
+        okt = __all_sync(0xffffffffu, okt);
+        if (!okt) return false;
         const float2 st = stats[t * BM + r];  // (1 / l, LSE)
         bar_arrive(stats_free(t));
-        ok = wait_bar(o_full(t), k & 1, ab, p.wait_ns, SITE_SOFT + 1);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
+        okt = wait_bar(o_full(t), k & 1, ab, p.wait_ns, SITE_SOFT + 1);
+        okt = __all_sync(0xffffffffu, okt);
+        if (!okt) return false;
         tc_fence_after();
         const float inv_l = st.x * o_mult;
         const uint32_t o_addr = tmem + lane_base + 256 + t * HD;
@@ -729,7 +737,70 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         }
         if (i < sv.len) p.lse[(size_t(sv.bt) * p.H + u.h) * (PACKED ? p.stat_rows : p.N) + sv.row0 + i] = st.y;
       }
+      return true;
+    };
+    // MASK_EPI: the keep bytes of block `kv0` (a local key index) of unit u
+    // for this thread's row of both tiles, into the next ring entry.  One
+    // generator call per quad of rows and 16 keys, shared through the quad
+    // (dropout_words_row16), the same draws the softmax would make itself.
+    int gm = 0;  // mask blocks written
+    auto write_mask = [&](const Unit& u, int kv0) -> bool {
+      const int m = gm % C::MASK_RING;
+      bool okm = wait_bar(mask_empty(m), ((gm / C::MASK_RING) & 1) ^ 1, ab, p.wait_ns, SITE_SOFT + 7);
+      okm = __all_sync(0xffffffffu, okm);
+      if (!okm) return false;
+      uint4* dst = sMask + m * (C::MASK_BYTES / 16);
+      const uint32_t thr4 = p.drop.threshold * 0x01010101u;
+      for (int t = 0; t < NQT; ++t) {
+        const int i = u.row0 + t * BM + r;
+#pragma unroll 2
+        for (int c = 0; c < BN / 16; ++c) {
+          uint32_t z[4];
+          dropout_words_row16(p.drop, u.b, u.h, i, (kv0 >> 2) + 4 * c, z);
+          dst[(t * (BN / 16) + c) * BM + r] = make_uint4(__vcmpgeu4(z[0], thr4), __vcmpgeu4(z[1], thr4),
+                                                         __vcmpgeu4(z[2], thr4), __vcmpgeu4(z[3], thr4));
+        }
+      }
+      bar_arrive(mask_full(m));
+      ++gm;
+      return true;
+    };
+    Unit prev{};
+    int kprev = -1;
+    for (int k = 0; ok; ++k) {
+      int L;
+      if (DYN) {
+        const int rr = k % C::RING;
+        ok = wait_bar(ring_full(rr), (k / C::RING) & 1, ab, p.wait_ns, SITE_SOFT + 3);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        L = ring[rr];
+        __syncwarp();
+        if (lane == 0) bar_arrive(ring_empty(rr));
+        if (L < 0) break;
+      } else {
+        L = unit_index(k);
+        if (L >= p.num_units) break;
+      }
+      const Unit u = unit_of<MODE>(p, L);
+      if (MASK_EPI) {
+        // The unit's first MASK_RING - 1 mask blocks go out before the
+        // previous unit's rows (the softmax starts this unit while they are
+        // stored), the rest after them: the previous unit's O must be read
+        // out of TMEM before this unit's first PV product, which waits on
+        // the softmax, which waits on these masks.
+        int kb = u.first, it = 0;
+        for (; ok && it < u.nblk && it < C::MASK_RING - 1; ++it, kb = next_block<MODE>(p, u, kb))
+          ok = write_mask(u, (SPARSE ? kb : u.first + it) * BN);
+        if (ok && kprev >= 0) ok = store_unit(prev, kprev);
+        for (; ok && it < u.nblk; ++it, kb = next_block<MODE>(p, u, kb))
+          ok = write_mask(u, (SPARSE ? kb : u.first + it) * BN);
+        prev = u;
+        kprev = k;
+      } else {
+        ok = store_unit(u, k);
+      }
     }
+    if (MASK_EPI && ok && kprev >= 0) store_unit(prev, kprev);
   } else {
     regs_inc<C::REGS_SOFT>();
     // ------------------------------------------------------------ softmax
@@ -848,7 +919,16 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
         // keeps the un-dropped sum and dropped probabilities leave P here:
         // one generator call per quad of rows and 16 keys (the rows of a quad
         // share i / 4: row0 is a multiple of 256), applied as 16-bit masks to
-        // the packed pairs.
+        // the packed pairs.  With MASK_EPI the epilogue warps have drawn the
+        // keep bytes into shared memory already.
+        const uint4* mask_row = nullptr;
+        if (MASK_EPI) {
+          const int gb = g + it;
+          ok = wait_bar(mask_full(gb % C::MASK_RING), (gb / C::MASK_RING) & 1, ab, p.wait_ns, SITE_SOFT + 8);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          mask_row = sMask + (gb % C::MASK_RING) * (C::MASK_BYTES / 16) + t * (BN / 16) * BM + r;
+        }
         if (FP8) {
           // e4m3 P: four per column, 32 columns.  P <= 2^TAU = 256 < 448.
 #pragma unroll
@@ -869,18 +949,29 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
           if (DROPOUT) {
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-              uint32_t z[4];
-              dropout_words_row16(p.drop, b, h, i, (kv0 >> 2) + 8 * c + 4 * half, z);
+              uint32_t km[4];  // keep bytes of keys kv0 + 32 c + 16 half + 4 g4 .. + 3
+              if (MASK_EPI) {
+                const uint4 w = mask_row[(2 * c + half) * BM];
+                km[0] = w.x;
+                km[1] = w.y;
+                km[2] = w.z;
+                km[3] = w.w;
+              } else {
+                uint32_t z[4];
+                dropout_words_row16(p.drop, b, h, i, (kv0 >> 2) + 8 * c + 4 * half, z);
+#pragma unroll
+                for (int g4 = 0; g4 < 4; ++g4) km[g4] = dropout_keep_bytes(z[g4], p.drop.threshold);
+              }
 #pragma unroll
               for (int g4 = 0; g4 < 4; ++g4) {
-                const uint32_t m = dropout_keep_bytes(z[g4], p.drop.threshold);
-                w16[8 * half + 2 * g4] &= __byte_perm(m, 0u, 0x1100);
-                w16[8 * half + 2 * g4 + 1] &= __byte_perm(m, 0u, 0x3322);
+                w16[8 * half + 2 * g4] &= __byte_perm(km[g4], 0u, 0x1100);
+                w16[8 * half + 2 * g4 + 1] &= __byte_perm(km[g4], 0u, 0x3322);
               }
             }
           }
           tmem_st16(p_addr + c * 16, w16);
         }
+        if (MASK_EPI) bar_arrive(mask_empty((g + it) % C::MASK_RING));  // its keep bytes are read
         // Rescale the running output (the PV product of the previous block has
         // completed: S_t of this block was committed after it, or, with the
         // separate-P layout, p_free said so).
