@@ -753,7 +753,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
       const uint32_t thr4 = p.drop.threshold * 0x01010101u;
       for (int t = 0; t < NQT; ++t) {
         const int i = u.row0 + t * BM + r;
-#pragma unroll 2
+#pragma unroll 4
         for (int c = 0; c < BN / 16; ++c) {
           uint32_t z[4];
           dropout_words_row16(p.drop, u.b, u.h, i, (kv0 >> 2) + 4 * c, z);
