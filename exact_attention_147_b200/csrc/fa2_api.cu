@@ -394,7 +394,7 @@ fa2_status launch_fwd_sm100(const AttnArgs& a, const fa2_strides& sq, const fa2_
   SchedLease lease;
   if (MODE != kLayoutPadded) FA2_TRY(lease.acquire(dev, device_info(dev), st, &p.sched));
   auto kern = fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, MODE, FP8>;
-  using Cfg = FwdCfg<HD, FP8, DROPOUT && HD == 128>;  // the kernel's own configuration
+  using Cfg = FwdKernelCfg<HD, DROPOUT, FP8>;  // the kernel's own configuration
   constexpr int smem = Cfg::SMEM_BYTES;
   FA2_TRY(ensure_smem(kern, smem, dev, mask));
   // The kernel re-balances registers between its warpgroups; the shares add

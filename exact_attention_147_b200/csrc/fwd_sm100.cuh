@@ -99,7 +99,7 @@ struct FwdCfg {
   static constexpr int BM = 128;        // query rows per tile
   static constexpr int BN = 128;        // keys per KV block
   static constexpr int NQT = 2;         // query tiles per unit
-  // MASK_EPI (d = 128 with dropout): the epilogue warps draw each block's
+  // MASK_EPI (the dropout kernels): the epilogue warps draw each block's
   // dropout mask into shared memory ahead of the softmax, in a ring of
   // MASK_RING blocks of keep bytes; Q is single-buffered to make room.
   static constexpr int QBUFS = MASK_EPI ? 1 : 2;  // Q buffers (across units)
@@ -132,11 +132,18 @@ struct FwdCfg {
   // (d = 64: 200 / 48 / 64 -- none of the roles spills, and the MMA issuer,
   // whose latency from a finished P to the next S product the softmax
   // waits on, measured about 1% faster with 64 than with 56)
-  static constexpr int REGS_SOFT = HD == 128 ? 184 : 200, REGS_EPI = HD == 128 ? 80 : 48,
+  // (d = 64 with the mask ring: 192 / 64 / 64, the epilogue runs the generator)
+  static constexpr int REGS_SOFT = HD == 128 ? 184 : (MASK_EPI ? 192 : 200),
+                       REGS_EPI = HD == 128 ? 80 : (MASK_EPI ? 64 : 48),
                        REGS_MISC = 64;
   static constexpr int REGS_AT_LAUNCH = (2 * 128 * REGS_SOFT + 128 * REGS_EPI + 128 * REGS_MISC) / 512;
   static_assert(REGS_AT_LAUNCH == 128, "register split must use exactly the launch budget");
 };
+
+// The configuration of fa2_fwd_sm100_kernel<HD, ALIBI, DROPOUT, MODE, FP8>:
+// the host sizes the launch (shared memory, registers) from the same type.
+template <int HD, bool DROPOUT, bool FP8>
+using FwdKernelCfg = FwdCfg<HD, FP8, DROPOUT>;
 
 namespace fwd_detail {
 constexpr float TAU = 8.0f;
@@ -273,9 +280,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 
 template <int HD, bool ALIBI, bool DROPOUT, int MODE, bool FP8 = false>
 __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
-  // d = 128 with dropout: the epilogue warps draw the mask (see FwdCfg)
-  constexpr bool MASK_EPI = DROPOUT && HD == 128;
-  using C = FwdCfg<HD, FP8, MASK_EPI>;
+  // with dropout the epilogue warps draw the mask (see FwdCfg)
+  constexpr bool MASK_EPI = DROPOUT;
+  using C = FwdKernelCfg<HD, DROPOUT, FP8>;
   static_assert(!FP8 || (HD == 128 && !DROPOUT && MODE == kLayoutPadded),
                 "e4m3 inputs: d = 128, padded layout, no dropout");
   constexpr int QBUFS = C::QBUFS;
@@ -321,8 +328,12 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
   // MASK_EPI: a block's keep bytes written by the epilogue / read by both softmax warpgroups
   auto mask_full = [&](int m) { return bar0 + 8u * (21 + 2 * SLOTS + 2 * C::RING + m); };
   auto mask_empty = [&](int m) { return bar0 + 8u * (21 + 2 * SLOTS + 2 * C::RING + C::MASK_RING + m); };
-  // [MASK_RING][NQT][BN / 16][BM] x 16 keep bytes (keys 16 c .. 16 c + 15 of one row)
+  // [MASK_RING][NQT][BN / 16][BM] x 16 keep bytes (keys 16 c .. 16 c + 15 of
+  // one row).  Within each 32 rows, row 4 m + w sits in slot 8 w + m, so that
+  // the writers (a quad of lanes holds rows 4 m .. 4 m + 3) store to 32
+  // different banks and every reader still takes one whole slot.
   uint4* sMask = reinterpret_cast<uint4*>(smem_raw + C::OFF_MASK);
+  auto mask_slot = [](int row) { return (row & ~31) | ((row & 3) << 3) | ((row >> 2) & 7); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* ring = abort_flag + 3;  // packed: unit indices handed from the producer to the other roles
@@ -740,25 +751,28 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
       return true;
     };
     // MASK_EPI: the keep bytes of block `kv0` (a local key index) of unit u
-    // for this thread's row of both tiles, into the next ring entry.  One
-    // generator call per quad of rows and 16 keys, shared through the quad
-    // (dropout_words_row16), the same draws the softmax would make itself.
+    // for both tiles, into the next ring entry: the same draws the softmax
+    // would make itself.  Lane s of a quad computes the generator call of
+    // key group 4 c + s for the quad's four rows (rows 4 (i / 4) .. + 3) and
+    // stores the four rows' words itself, so no lane needs the others' words.
     int gm = 0;  // mask blocks written
     auto write_mask = [&](const Unit& u, int kv0) -> bool {
       const int m = gm % C::MASK_RING;
       bool okm = wait_bar(mask_empty(m), ((gm / C::MASK_RING) & 1) ^ 1, ab, p.wait_ns, SITE_SOFT + 7);
       okm = __all_sync(0xffffffffu, okm);
       if (!okm) return false;
-      uint4* dst = sMask + m * (C::MASK_BYTES / 16);
+      const int s4 = lane & 3;
+      // word s4 of the slots of rows 4 (r / 4) + w, w = 0..3 (slot 8 w + r / 4 mod 8)
+      uint32_t* dst = reinterpret_cast<uint32_t*>(sMask + m * (C::MASK_BYTES / 16)) +
+                      (mask_slot(r & ~3)) * 4 + s4;
       const uint32_t thr4 = p.drop.threshold * 0x01010101u;
       for (int t = 0; t < NQT; ++t) {
-        const int i = u.row0 + t * BM + r;
+        const uint32_t i4 = uint32_t((u.row0 + t * BM + r) >> 2);
 #pragma unroll 4
         for (int c = 0; c < BN / 16; ++c) {
-          uint32_t z[4];
-          dropout_words_row16(p.drop, u.b, u.h, i, (kv0 >> 2) + 4 * c, z);
-          dst[(t * (BN / 16) + c) * BM + r] = make_uint4(__vcmpgeu4(z[0], thr4), __vcmpgeu4(z[1], thr4),
-                                                         __vcmpgeu4(z[2], thr4), __vcmpgeu4(z[3], thr4));
+          const Philox4 o = philox4x32_10(uint32_t((kv0 >> 2) + 4 * c + s4), i4, uint32_t(u.h), uint32_t(u.b), p.drop);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) dst[((t * (BN / 16) + c) * BM + 8 * w) * 4] = __vcmpgeu4(o.w[w], thr4);
         }
       }
       bar_arrive(mask_full(m));
@@ -927,7 +941,7 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
           ok = wait_bar(mask_full(gb % C::MASK_RING), (gb / C::MASK_RING) & 1, ab, p.wait_ns, SITE_SOFT + 8);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          mask_row = sMask + (gb % C::MASK_RING) * (C::MASK_BYTES / 16) + t * (BN / 16) * BM + r;
+          mask_row = sMask + (gb % C::MASK_RING) * (C::MASK_BYTES / 16) + t * (BN / 16) * BM + mask_slot(r);
         }
         if (FP8) {
           // e4m3 P: four per column, 32 columns.  P <= 2^TAU = 256 < 448.
