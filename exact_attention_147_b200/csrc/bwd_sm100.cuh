@@ -703,9 +703,9 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
             dropout_words_col16(p.drop, b, h, j, (i0 >> 2) + 4 * t16, z);
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
-              // 0xFF in each kept byte, then the bytes' top bits gathered into
-              // bits 28..31 by one multiply (the shifted copies never overlap)
-              const uint32_t m = dropout_keep_bytes(z[c4], p.drop.threshold) & 0x80808080u;
+              // bit 7 of each kept byte, the four gathered into bits 28..31
+              // by one multiply (the shifted copies never overlap)
+              const uint32_t m = dropout_keep_msb4(z[c4], p.drop.threshold);
               const uint32_t nib = (m * 0x00204081u) >> 28;  // bit e: query 4 c4 + e kept
               const int c = 16 * t16 + 4 * c4;
               if (c < 32) keep_lo |= nib << c;

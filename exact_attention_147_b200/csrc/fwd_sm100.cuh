@@ -765,14 +765,14 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
       // word s4 of the slots of rows 4 (r / 4) + w, w = 0..3 (slot 8 w + r / 4 mod 8)
       uint32_t* dst = reinterpret_cast<uint32_t*>(sMask + m * (C::MASK_BYTES / 16)) +
                       (mask_slot(r & ~3)) * 4 + s4;
-      const uint32_t thr4 = p.drop.threshold * 0x01010101u;
       for (int t = 0; t < NQT; ++t) {
         const uint32_t i4 = uint32_t((u.row0 + t * BM + r) >> 2);
 #pragma unroll 4
         for (int c = 0; c < BN / 16; ++c) {
           const Philox4 o = philox4x32_10(uint32_t((kv0 >> 2) + 4 * c + s4), i4, uint32_t(u.h), uint32_t(u.b), p.drop);
 #pragma unroll
-          for (int w = 0; w < 4; ++w) dst[((t * (BN / 16) + c) * BM + 8 * w) * 4] = __vcmpgeu4(o.w[w], thr4);
+          for (int w = 0; w < 4; ++w)
+            dst[((t * (BN / 16) + c) * BM + 8 * w) * 4] = dropout_keep_msb4(o.w[w], p.drop.threshold);
         }
       }
       bar_arrive(mask_full(m));
@@ -930,11 +930,10 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
           tc_fence_after();
         }
         // P (bf16 pairs) over the first BN/2 columns of S.  With dropout, l
-        // keeps the un-dropped sum and dropped probabilities leave P here:
-        // one generator call per quad of rows and 16 keys (the rows of a quad
-        // share i / 4: row0 is a multiple of 256), applied as 16-bit masks to
-        // the packed pairs.  With MASK_EPI the epilogue warps have drawn the
-        // keep bytes into shared memory already.
+        // keeps the un-dropped sum and dropped probabilities leave P here: the
+        // epilogue warps have drawn the keep bits (bit 7 of each key's byte)
+        // into shared memory, and each pair's two bits become 16-bit masks by
+        // sign-replicating byte permutes.
         const uint4* mask_row = nullptr;
         if (MASK_EPI) {
           const int gb = g + it;
@@ -963,23 +962,13 @@ __global__ void __launch_bounds__(512, 1) fa2_fwd_sm100_kernel(const __grid_cons
           if (DROPOUT) {
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-              uint32_t km[4];  // keep bytes of keys kv0 + 32 c + 16 half + 4 g4 .. + 3
-              if (MASK_EPI) {
-                const uint4 w = mask_row[(2 * c + half) * BM];
-                km[0] = w.x;
-                km[1] = w.y;
-                km[2] = w.z;
-                km[3] = w.w;
-              } else {
-                uint32_t z[4];
-                dropout_words_row16(p.drop, b, h, i, (kv0 >> 2) + 8 * c + 4 * half, z);
-#pragma unroll
-                for (int g4 = 0; g4 < 4; ++g4) km[g4] = dropout_keep_bytes(z[g4], p.drop.threshold);
-              }
+              // keep bits of keys kv0 + 32 c + 16 half + 4 g4 .. + 3, as bit 7 of each byte
+              const uint4 w = mask_row[(2 * c + half) * BM];
+              const uint32_t km[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
               for (int g4 = 0; g4 < 4; ++g4) {
-                w16[8 * half + 2 * g4] &= __byte_perm(km[g4], 0u, 0x1100);
-                w16[8 * half + 2 * g4 + 1] &= __byte_perm(km[g4], 0u, 0x3322);
+                w16[8 * half + 2 * g4] &= prmt(km[g4], 0u, 0x9988);
+                w16[8 * half + 2 * g4 + 1] &= prmt(km[g4], 0u, 0xBBAA);
               }
             }
           }

@@ -124,9 +124,14 @@ __device__ __forceinline__ void dropout_words_col16(const DropoutParams& dp, int
   quad_transpose(x, z);
 }
 
-// 0xFF in every byte of `word` that is kept (byte >= threshold), else 0x00.
-__device__ __forceinline__ uint32_t dropout_keep_bytes(uint32_t word, uint32_t threshold) {
-  return __vcmpgeu4(word, threshold * 0x01010101u);
+// 0x80 in every byte of `word` that is kept (byte >= threshold t), else 0x00,
+// in three integer operations: d = (word | 0x80808080) - (t mod 128) * 0x01010101
+// cannot borrow across bytes, and bit 7 of a byte of d says whether that
+// byte's low seven bits are >= those of t; so the byte is >= t iff its bit 7
+// or d's is set (t < 128), or both are (t >= 128).
+__device__ __forceinline__ uint32_t dropout_keep_msb4(uint32_t word, uint32_t threshold) {
+  const uint32_t d = (word | 0x80808080u) - (threshold & 0x7Fu) * 0x01010101u;
+  return (threshold < 128u ? (word | d) : (word & d)) & 0x80808080u;
 }
 
 // Byte e (0..3) of a packed word kept?
