@@ -20,7 +20,7 @@ from exact_attention_147_b200 import fa2 as F
 from exact_attention_147_b200 import workloads as W
 from oracle import attention as oa
 from oracle import philox
-from tests.helpers import check_fwd, check_grad, f64
+from tests.helpers import assert_same_sum_any_order, check_fwd, check_grad, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +36,7 @@ def onehot_half(n, d, half, dtype):
 
 @pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("p,seed", [(0.5, 11), (0.1, 2**40 + 7)])
+@pytest.mark.parametrize("p,seed", [(0.5, 11), (0.1, 2**40 + 7), (0.99, 5)])
 def test_mask_bits_forward_and_backward(dtype, p, seed, d):
     B, N, H = 2, 256, 3
     q = torch.zeros(B, N, H, d, dtype=dtype, device="cuda")
@@ -145,3 +145,22 @@ def test_autograd_draws_fresh_masks():
     qg = q.clone().requires_grad_(True)
     F.flash_attention_v2(qg, k, v, dropout_p=0.3).backward(do)
     assert torch.isfinite(qg.grad).all()
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_threshold_zero_keeps_everything(d):
+    # p < 0.5/256 rounds the byte threshold to 0: every byte passes and the
+    # keep scale is 256/256, so the dropout kernels must give exactly what
+    # the kernels without dropout give.
+    w = W.Workload("drop-t0", B=1, N=384, H=2, d=d, causal=True, seed=57)
+    q, k, v, do = W.make_inputs(w, "cuda")
+    ref = F.fwd(q, k, v, causal=True)
+    got = F.fwd(q, k, v, causal=True, dropout_p=1e-3, dropout_seed=3)
+    D = F.bwd_preprocess(ref[0], do)
+    gref = F.bwd(do, q, k, v, ref[1], D, causal=True)
+    ggot = F.bwd(do, q, k, v, ref[1], D, causal=True, dropout_p=1e-3, dropout_seed=3)
+    torch.cuda.synchronize()
+    assert F.device_status() == 0
+    assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
+    for a, b in zip(ggot, gref):
+        assert_same_sum_any_order(a, b)
