@@ -12,7 +12,9 @@
 // Inside a CTA (16 warps, four warpgroups):
 //   warps 0-3   softmax for query tile 0 (thread = one query row)
 //   warps 4-7   softmax for query tile 1
-//   warps 8-11  epilogue: O_t / l out of TMEM, bf16 rows and LSE to HBM
+//   warps 8-11  epilogue: O_t / l out of TMEM, bf16 rows and LSE to HBM;
+//               with dropout they also draw each block's mask (keep bits)
+//               into a shared-memory ring a block ahead of the softmax
 //   warp  12    TMA producer: Q once per unit, then K_j, V_j into a ring of slots
 //   warp  13    MMA issuer: S_t = Q_t K_j^T and O_t += P_t V_j (tcgen05)
 //   warps 14-15 idle (they complete the fourth warpgroup for setmaxnreg)
@@ -20,9 +22,10 @@
 // multi-slot TMA + mbarrier ring ("FlashAttention v2" article, §3.1-§3.2:
 // Q kept on chip, K/V prefetched while the current block is computed).
 //
-// The Q buffers are double-buffered across units; O leaves through registers
+// The Q buffers are double-buffered across units (single-buffered with
+// dropout, whose mask ring takes that space); O leaves through registers
 // (normalised, cast to bf16 and stored by the row's own thread), so shared
-// memory holds only Q and the K/V ring.
+// memory holds only Q, the K/V ring and, with dropout, the mask ring.
 //
 // Tensor memory (512 columns x 128 lanes of fp32):
 //   [0,128)    S_0 (P_0 as bf16 pairs in its first 64 columns)
