@@ -71,11 +71,15 @@ KERNEL_SOURCES = {
 
 
 def sources_hash(call):
+    """Hash of the kernel sources with their // comments and blank lines
+    removed, so that a comment-only edit keeps a capture valid."""
     import hashlib
+    import re
     m = hashlib.sha256()
     for f in sorted(KERNEL_SOURCES[call]):
-        with open(os.path.join(ROOT, "exact_attention_147_b200", "csrc", f), "rb") as fh:
-            m.update(fh.read())
+        with open(os.path.join(ROOT, "exact_attention_147_b200", "csrc", f), encoding="utf-8") as fh:
+            code = [re.sub(r"//.*$", "", ln).rstrip() for ln in fh.read().splitlines()]
+        m.update("\n".join(ln for ln in code if ln).encode())
     return m.hexdigest()[:16]
 
 
