@@ -88,11 +88,16 @@ struct BwdCfg {
   static constexpr int OFF_SIDE = OFF_DS + DS_BYTES;
   static constexpr int OFF_STG = OFF_SIDE + Q_STAGES * SIDE_BYTES;  // dQ staging ring
   static constexpr int STG_BYTES = 2 * 16384;                         // 2 x (128 rows x 32 fp32)
-  static constexpr int OFF_BARS = OFF_STG + STG_BYTES;
+  // d = 64 has room for a second K, V pair: the next item's K and V load
+  // while the current item runs (d = 128 fills shared memory with one pair)
+  static constexpr int KV_BUFS = HD == 64 ? 2 : 1;
+  static constexpr int OFF_KV2 = OFF_STG + STG_BYTES;
+  static constexpr int OFF_BARS = OFF_KV2 + (KV_BUFS - 1) * 2 * TILE;
   static constexpr int RING = 4;                      // item-index ring (packed / block-sparse)
   // kv_full, Q full/empty, dO full/empty, s_full, dp_full, p_ready, ds_ready,
-  // dq_full, dq_free, acc_full, drain, kv_empty, acc_empty, ring full/empty
-  static constexpr int NBARS = 1 + 2 * Q_STAGES + 2 * DO_STAGES + 8 + 2 + 2 * RING;
+  // dq_full, dq_free, acc_full, drain, kv_empty, acc_empty, ring full/empty,
+  // then kv_full / kv_empty of the second K, V pair
+  static constexpr int NBARS = 1 + 2 * Q_STAGES + 2 * DO_STAGES + 8 + 2 + 2 * RING + 2 * (KV_BUFS - 1);
   // No alignment slack: the kernel checks that the dynamic shared memory
   // starts on a 1024-byte boundary (it does: the reserved 1 KB precedes it).
   // barriers, then the TMEM address, the abort flag, 2 spare words, the ring
@@ -296,6 +301,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   constexpr bool PACKED = MODE == kLayoutPacked;
   constexpr bool SPARSE = MODE == kLayoutSparse;
   constexpr bool DYN = PACKED || SPARSE || DSCHED;  // items taken from the shared counter
+  // K, V pairs in use: the counter-scheduled calls keep one, so that a CTA
+  // claims its next item only once its current item's K and V are free (a
+  // second pair let CTAs claim a whole item earlier, which unbalanced the
+  // end of long causal calls: d = 64, N = 16384, -8%)
+  constexpr int KVB = DYN ? 1 : C::KV_BUFS;
   using namespace bwd_detail;
   constexpr int QS = C::Q_STAGES, DS = C::DO_STAGES;
   // Register split.  The ordered dQ's drain holds a whole 128-column fp32
@@ -328,7 +338,6 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   float* sSide = reinterpret_cast<float*>(smem + C::OFF_SIDE);  // [QS][2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t kv_full = b0;
   auto q_full = [&](int s) { return b0 + 8u * (1 + s); };
   auto q_empty = [&](int s) { return b0 + 8u * (1 + QS + s); };
   auto do_full = [&](int s) { return b0 + 8u * (1 + 2 * QS + s); };
@@ -337,7 +346,12 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
   const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24;
   const uint32_t dq_full = s_full + 32, dq_free = s_full + 40, acc_full = s_full + 48;
   const uint32_t drain_bar = s_full + 56;
-  const uint32_t kv_empty = s_full + 64, acc_empty = s_full + 72;
+  const uint32_t acc_empty = s_full + 72;
+  // K, V buffer pair b and its barriers (pair 1 after the ring's barriers)
+  auto kv_full = [&](int b) { return b == 0 ? b0 : s_full + 80 + 16u * C::RING; };
+  auto kv_empty = [&](int b) { return b == 0 ? s_full + 64 : s_full + 88 + 16u * C::RING; };
+  auto kv_k = [&](int b) { return b == 0 ? sK : smem + C::OFF_KV2; };
+  auto kv_v = [&](int b) { return b == 0 ? sV : smem + C::OFF_KV2 + C::TILE; };
   auto ring_full = [&](int r) { return s_full + 80 + 8u * r; };
   auto ring_empty = [&](int r) { return s_full + 80 + 8u * (C::RING + r); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
@@ -425,15 +439,19 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         }
         const BItem itm = item_of<MODE, ORDER>(p, I);
         int I_next = 0;
-        // K and V of this item once the previous item's products have read them
-        ok = wait_bar(kv_empty, (jn & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 2);
+        // K and V of this item once the products of the item that last used
+        // this buffer pair have read them
+        const int kvb = jn % KVB;
+        ok = wait_bar(kv_empty(kvb), ((jn / KVB) & 1) ^ 1, ab, p.wait_ns, SITE_BPROD + 2);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         if (lane == 0) {
-          bar_arrive_expect_tx(kv_full, 2 * C::TILE);
+          bar_arrive_expect_tx(kv_full(kvb), 2 * C::TILE);
           for (int c = 0; c < NCH; ++c) {
-            tma_load_4d(smem_u32(sK + c * 16384), &p.tm_k, kv_full, c * 64, itm.h, itm.trow + itm.k0, itm.bt);
-            tma_load_4d(smem_u32(sV + c * 16384), &p.tm_v, kv_full, c * 64, itm.h, itm.trow + itm.k0, itm.bt);
+            tma_load_4d(smem_u32(kv_k(kvb) + c * 16384), &p.tm_k, kv_full(kvb), c * 64, itm.h,
+                        itm.trow + itm.k0, itm.bt);
+            tma_load_4d(smem_u32(kv_v(kvb) + c * 16384), &p.tm_v, kv_full(kvb), c * 64, itm.h,
+                        itm.trow + itm.k0, itm.bt);
           }
         }
         ++issued_kv;
@@ -501,7 +519,8 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       // The last CTA to finish taking items returns the counters to zero.
       if (DYN && lane == 0) sched_cta_done(p.sched);
       if (lane == 0) {  // every copy issued must land before the CTA exits
-        if (issued_kv > 0) drain_wait(kv_full, (issued_kv - 1) & 1, p.wait_ns);
+        for (int j = max(0, issued_kv - KVB); j < issued_kv; ++j)
+          drain_wait(kv_full(j % KVB), (j / KVB) & 1, p.wait_ns);
         for (int q = max(0, issued_q - QS); q < issued_q; ++q)
           drain_wait(q_full(q % QS), (q / QS) & 1, p.wait_ns);
         for (int q = max(0, issued_do - DS); q < issued_do; ++q)
@@ -537,13 +556,15 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
       //   S_{i+2}          (S columns are free once dV_{i+1} has read P_{i+1})
       // The compute warps work in the order P_0, dS_0, P_1, dS_1, ...
       // Indices below are the CTA-wide query-block counter g + i.
+      const uint8_t* curK = sK;  // this item's K and V
+      const uint8_t* curV = sV;
       auto dp = [&](int k) {                      // dP_k^T = V dO_k^T
         const int sd = k % DS;
         if (!wait_bar(do_full(sd), (k / DS) & 1, ab, p.wait_ns, SITE_BMMA + 2)) return false;
         if (WITH_DQ && k > 0 && !wait_bar(dq_free, (k - 1) & 1, ab, p.wait_ns, SITE_BMMA + 3))
           return false;
         tc_fence_after();
-        kmajor(tmem + T_DP, sV, sDO + sd * C::TILE);
+        kmajor(tmem + T_DP, curV, sDO + sd * C::TILE);
         umma_commit(dp_full);
         return true;
       };
@@ -559,7 +580,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         const int sn = k % QS;
         if (!wait_bar(q_full(sn), (k / QS) & 1, ab, p.wait_ns, SITE_BMMA + 5)) return false;
         tc_fence_after();
-        kmajor(tmem + T_S, sK, sQ + sn * C::TILE);
+        kmajor(tmem + T_S, curK, sQ + sn * C::TILE);
         umma_commit(s_full);
         return true;
       };
@@ -573,8 +594,11 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
         if (!ok || I < 0) break;
         const BItem itm = item_of<MODE, ORDER>(p, I);
         const int nq = itm.nq;
+        const int kvb = jn % KVB;
+        curK = kv_k(kvb);
+        curV = kv_v(kvb);
         if (lane == 0) {
-          ok = wait_bar(kv_full, jn & 1, ab, p.wait_ns, SITE_BMMA + 0);
+          ok = wait_bar(kv_full(kvb), (jn / KVB) & 1, ab, p.wait_ns, SITE_BMMA + 0);
           ok = ok && s_next(g);
           ok = ok && dp(g);
           // dV_0 and dK_0 overwrite the accumulators: the compute warps must
@@ -593,7 +617,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
             if (WITH_DQ) {
               // dQ_i = dS K: A = dS (queries x keys) read MN-major from the
               // dS^T tile, B = K (keys x d) MN-major.
-              const uint32_t a0 = smem_u32(sDS), kb0 = smem_u32(sK);
+              const uint32_t a0 = smem_u32(sDS), kb0 = smem_u32(curK);
 #pragma unroll
               for (int kk = 0; kk < 128 / 16; ++kk)
                 umma_ss(tmem + T_DP, sdesc_sw128(a0 + kk * 2048, 16384, 1024),
@@ -604,7 +628,7 @@ __global__ void __launch_bounds__(512, 1) fa2_bwd_dkdv_sm100_kernel(const __grid
             if (ok && it + 2 < nq) ok = s_next(gi + 2);
           }
           if (ok) {
-            umma_commit(kv_empty);   // every product reading K and V is issued
+            umma_commit(kv_empty(kvb));   // every product reading K and V is issued
             umma_commit(acc_full);
           }
         }
