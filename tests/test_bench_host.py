@@ -78,3 +78,19 @@ def test_reference_arm_prints_the_gpu_arms_config(monkeypatch, capsys):
     assert 0 < line["ms_per_step"] < line["ms_per_full_step_extrapolated"]
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_traffic_key_ignores_comments_only(tmp_path, monkeypatch):
+    # the committed capture stays valid across a comment-only edit of the
+    # kernel sources, and not across a change of code
+    import shutil
+    src = os.path.join(ROOT, "exact_attention_147_b200", "csrc")
+    dst = tmp_path / "exact_attention_147_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    before = bench.sources_hash("fa2_bwd")
+    f = dst / "bwd_sm100.cuh"
+    f.write_text(f.read_text() + "\n// a note\n\n")
+    assert bench.sources_hash("fa2_bwd") == before
+    f.write_text(f.read_text() + "\nstatic const int unused_probe_constant = 1;\n")
+    assert bench.sources_hash("fa2_bwd") != before
